@@ -1,0 +1,423 @@
+// C-ABI entry points of libmimoattn: host-side validation, TMA descriptors,
+// workspace carving and kernel dispatch.  See include/mimoattn.h for the
+// contract of each call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mimoattn.h"
+#include "internal.h"
+
+namespace mimo {
+
+__device__ unsigned g_status_word;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+#define REQUIRE_PTR(p, name)                                                                        \
+  do {                                                                                              \
+    if ((p) == nullptr) return fail(MIMO_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);             \
+    if (!aligned16(p)) return fail(MIMO_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, name); \
+  } while (0)
+
+int check_layer(const char* fn, const mimo_layer& L) {
+  if (L.num_q_heads != kHq || L.head_dim_qk != kDqk || L.head_dim_v != kDv || L.rope_dim != kRope)
+    return fail(MIMO_ERR_UNSUPPORTED, "%s: only 64 query heads, head dims 192/128 and rope_dim 64 are supported", fn);
+  if (L.num_kv_heads != 8 && L.num_kv_heads != 4)
+    return fail(MIMO_ERR_UNSUPPORTED, "%s: num_kv_heads must be 8 or 4 (got %d)", fn, L.num_kv_heads);
+  if (!(L.rope_base > 0.0) || !std::isfinite(L.rope_base))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: rope_base must be a finite positive number", fn);
+  if (!(L.softmax_scale > 0.f) || !std::isfinite(L.softmax_scale))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: softmax_scale must be finite and positive", fn);
+  if (!std::isfinite(L.v_scale)) return fail(MIMO_ERR_INVALID_ARG, "%s: v_scale must be finite", fn);
+  if (L.window < 0) return fail(MIMO_ERR_INVALID_ARG, "%s: window must be >= 0", fn);
+  if (L.sink && (reinterpret_cast<uintptr_t>(L.sink) & 3))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: sink is not 4-byte aligned", fn);
+  return MIMO_OK;
+}
+
+RopeFreqs make_freqs(double base) {
+  RopeFreqs f;
+  for (int j = 0; j < kHalf; ++j) f.inv_freq[j] = std::pow(base, -2.0 * double(j) / double(kRope));
+  return f;
+}
+
+// Per-device state: address of the status word and the SM count.
+struct DevState {
+  unsigned* status = nullptr;
+  int sms = 0;
+};
+std::mutex g_mu;
+DevState g_dev[64];
+
+int dev_state(const char* fn, DevState* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(MIMO_ERR_CUDA, "%s: device index %d out of range", fn, dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState& d = g_dev[dev];
+  if (!d.status) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_status_word);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress: %s", fn, cudaGetErrorString(e));
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaDeviceGetAttribute: %s", fn, cudaGetErrorString(e));
+    d.status = static_cast<unsigned*>(ptr);
+  }
+  *out = d;
+  return MIMO_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(const char* fn, EncodeTiledFn* out) {
+  static EncodeTiledFn enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  if (!enc) return fail(MIMO_ERR_CUDA, "%s: cuTensorMapEncodeTiled is not available", fn);
+  *out = enc;
+  return MIMO_OK;
+}
+
+// 3-D bf16 tensor [rows, heads, dim] (dim innermost) with box {64, box_h, box_rows},
+// 128-byte swizzle, zero fill out of bounds.
+int make_map(const char* fn, EncodeTiledFn enc, CUtensorMap* m, const void* base, long rows, int heads, int dim,
+             int box_h, int box_rows) {
+  cuuint64_t gdim[3] = {cuuint64_t(dim), cuuint64_t(heads), cuuint64_t(rows < 1 ? 1 : rows)};
+  cuuint64_t gstride[2] = {cuuint64_t(dim) * 2, cuuint64_t(dim) * 2 * heads};
+  cuuint32_t box[3] = {64, cuuint32_t(box_h), cuuint32_t(box_rows)};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MIMO_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", fn, int(r));
+  return MIMO_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int decode_split_len(int max_seq_len, int window) {
+  const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
+  if (n <= 256) return 256;
+  return 512;
+}
+
+}  // namespace
+}  // namespace mimo
+
+using namespace mimo;
+
+extern "C" {
+
+const char* mimo_last_error(void) { return g_err; }
+
+const char* mimo_version(void) { return "libmimoattn 0.1 (sm_100a)"; }
+
+size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_k, int num_kv_heads, int cache_kind) {
+  if (num_seqs < 0 || total_k < 0 || num_kv_heads <= 0) return 0;
+  if (cache_kind == MIMO_CACHE_PAGED) return 0;
+  if (cache_kind == MIMO_CACHE_RING) {
+    const size_t rows = size_t(total_k) + 128 * size_t(num_seqs);
+    return round256(rows * num_kv_heads * kDqk * 2) + round256(rows * num_kv_heads * kDv * 2);
+  }
+  return round256(size_t(total_k) * num_kv_heads * kRope * 2);
+}
+
+size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int num_kv_heads, int window) {
+  (void)num_kv_heads;
+  if (batch <= 0 || max_seq_len <= 0) return 0;
+  const int split = decode_split_len(max_seq_len, window);
+  const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
+  const int ns = (n + split - 1) / split;
+  if (ns <= 1) return 0;
+  return round256(size_t(batch) * kHq * ns * kDv * 4) + round256(size_t(batch) * kHq * ns * 2 * 4);
+}
+
+int mimo_kv_append(const mimo_append_args* a, void* stream) {
+  const char* fn = "mimo_kv_append";
+  if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->head_dim_qk != kDqk || a->head_dim_v != kDv || a->rope_dim != kRope)
+    return fail(MIMO_ERR_UNSUPPORTED, "%s: only head dims 192/128 and rope_dim 64 are supported", fn);
+  if (a->num_kv_heads != 8 && a->num_kv_heads != 4)
+    return fail(MIMO_ERR_UNSUPPORTED, "%s: num_kv_heads must be 8 or 4", fn);
+  if (!(a->rope_base > 0.0) || !std::isfinite(a->rope_base))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: rope_base must be a finite positive number", fn);
+  if (a->num_tokens < 0) return fail(MIMO_ERR_INVALID_ARG, "%s: num_tokens must be >= 0", fn);
+  if (a->cache_kind != MIMO_CACHE_RING && a->cache_kind != MIMO_CACHE_PAGED)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: cache_kind must be MIMO_CACHE_RING or MIMO_CACHE_PAGED", fn);
+  if (a->num_seqs <= 0) return fail(MIMO_ERR_INVALID_ARG, "%s: num_seqs must be > 0", fn);
+  if (a->num_tokens == 0) return MIMO_OK;
+  REQUIRE_PTR(a->k_new, "k_new");
+  REQUIRE_PTR(a->v_new, "v_new");
+  REQUIRE_PTR(a->pos, "pos");
+  REQUIRE_PTR(a->seq_idx, "seq_idx");
+  REQUIRE_PTR(a->k_cache, "k_cache");
+  REQUIRE_PTR(a->v_cache, "v_cache");
+  if (a->cache_kind == MIMO_CACHE_PAGED) {
+    REQUIRE_PTR(a->block_table, "block_table");
+    if (a->max_pages <= 0 || a->num_pages <= 0)
+      return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages and num_pages must be > 0 for a paged cache", fn);
+  }
+  DevState d;
+  if (int rc = dev_state(fn, &d)) return rc;
+  AppendParams p;
+  p.num_tokens = a->num_tokens;
+  p.hkv = a->num_kv_heads;
+  p.k_new = static_cast<const uint16_t*>(a->k_new);
+  p.v_new = static_cast<const uint16_t*>(a->v_new);
+  p.pos = a->pos;
+  p.seq_idx = a->seq_idx;
+  p.cache_kind = a->cache_kind;
+  p.k_cache = static_cast<uint16_t*>(a->k_cache);
+  p.v_cache = static_cast<uint16_t*>(a->v_cache);
+  p.num_seqs = a->num_seqs;
+  p.block_table = a->block_table;
+  p.max_pages = a->max_pages;
+  p.num_pages = a->num_pages;
+  p.rope = make_freqs(a->rope_base);
+  p.status = d.status;
+  cudaError_t e = launch_kv_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return MIMO_OK;
+}
+
+int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
+  const char* fn = "mimo_attn_decode";
+  if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (int rc = check_layer(fn, a->layer)) return rc;
+  if (a->batch < 0) return fail(MIMO_ERR_INVALID_ARG, "%s: batch must be >= 0", fn);
+  if (a->batch == 0) return MIMO_OK;
+  if (a->max_seq_len <= 0) return fail(MIMO_ERR_INVALID_ARG, "%s: max_seq_len must be > 0", fn);
+  if (a->cache_kind != MIMO_CACHE_RING && a->cache_kind != MIMO_CACHE_PAGED)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: cache_kind must be MIMO_CACHE_RING or MIMO_CACHE_PAGED", fn);
+  if (a->cache_kind == MIMO_CACHE_RING && (a->layer.window <= 0 || a->layer.window > 128))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: a ring cache holds 128 positions: window must be in 1..128", fn);
+  REQUIRE_PTR(a->q, "q");
+  REQUIRE_PTR(a->seq_lens, "seq_lens");
+  REQUIRE_PTR(a->k_cache, "k_cache");
+  REQUIRE_PTR(a->v_cache, "v_cache");
+  REQUIRE_PTR(a->out, "out");
+  if (a->lse && (reinterpret_cast<uintptr_t>(a->lse) & 3))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: lse is not 4-byte aligned", fn);
+  if (a->cache_kind == MIMO_CACHE_PAGED) {
+    REQUIRE_PTR(a->block_table, "block_table");
+    if (a->max_pages <= 0 || a->num_pages <= 0)
+      return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages and num_pages must be > 0 for a paged cache", fn);
+    if (long(a->max_pages) * kPage < a->max_seq_len)
+      return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages * 128 is below max_seq_len", fn);
+  }
+  const size_t need = mimo_attn_decode_workspace_size(a->batch, a->max_seq_len, a->layer.num_kv_heads, a->layer.window);
+  if (need > 0) {
+    if (!a->workspace || a->workspace_bytes < need)
+      return fail(MIMO_ERR_WORKSPACE, "%s: workspace of %zu bytes required (got %zu)", fn, need,
+                  a->workspace ? a->workspace_bytes : size_t(0));
+    if (!aligned16(a->workspace)) return fail(MIMO_ERR_INVALID_ARG, "%s: workspace is not 16-byte aligned", fn);
+  }
+  DevState d;
+  if (int rc = dev_state(fn, &d)) return rc;
+  DecodeParams p;
+  p.batch = a->batch;
+  p.hkv = a->layer.num_kv_heads;
+  p.group = kHq / p.hkv;
+  p.window = a->layer.window;
+  p.split_len = decode_split_len(a->max_seq_len, a->layer.window);
+  const int n = p.window > 0 ? (a->max_seq_len < p.window ? a->max_seq_len : p.window) : a->max_seq_len;
+  p.max_splits = (n + p.split_len - 1) / p.split_len;
+  p.scale_log2 = a->layer.softmax_scale * 1.4426950408889634f;
+  p.v_scale = a->layer.v_scale;
+  p.sink = a->layer.sink;
+  p.q = static_cast<const uint16_t*>(a->q);
+  p.seq_lens = a->seq_lens;
+  p.cache_kind = a->cache_kind;
+  p.k_cache = static_cast<const uint16_t*>(a->k_cache);
+  p.v_cache = static_cast<const uint16_t*>(a->v_cache);
+  p.block_table = a->block_table;
+  p.max_pages = a->max_pages;
+  p.num_pages = a->num_pages;
+  p.out = static_cast<uint16_t*>(a->out);
+  p.lse = a->lse;
+  p.ws_o = need ? static_cast<float*>(a->workspace) : nullptr;
+  p.ws_ml = need ? reinterpret_cast<float*>(static_cast<char*>(a->workspace) +
+                                            round256(size_t(a->batch) * kHq * p.max_splits * kDv * 4))
+                 : nullptr;
+  p.rope = make_freqs(a->layer.rope_base);
+  p.status = d.status;
+  cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return MIMO_OK;
+}
+
+int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
+  const char* fn = "mimo_attn_prefill";
+  if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (int rc = check_layer(fn, a->layer)) return rc;
+  if (a->num_seqs <= 0) return fail(MIMO_ERR_INVALID_ARG, "%s: num_seqs must be > 0", fn);
+  if (a->total_q < 0 || a->total_k < 0) return fail(MIMO_ERR_INVALID_ARG, "%s: total_q/total_k must be >= 0", fn);
+  if (a->cache_kind != MIMO_CACHE_NONE && a->cache_kind != MIMO_CACHE_RING && a->cache_kind != MIMO_CACHE_PAGED)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: unknown cache_kind %d", fn, a->cache_kind);
+  if (a->total_q == 0) return MIMO_OK;
+  REQUIRE_PTR(a->q, "q");
+  REQUIRE_PTR(a->out, "out");
+  REQUIRE_PTR(a->cu_seqlens_q, "cu_seqlens_q");
+  if (a->lse && (reinterpret_cast<uintptr_t>(a->lse) & 3))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: lse is not 4-byte aligned", fn);
+  const int hkv = a->layer.num_kv_heads;
+  int mode;
+  if (a->cache_kind == MIMO_CACHE_PAGED) {
+    if (a->k || a->v || a->cu_seqlens_k || a->total_k)
+      return fail(MIMO_ERR_INVALID_ARG,
+                  "%s: with a paged cache all keys come from the cache (append them first); k, v, cu_seqlens_k "
+                  "must be NULL and total_k 0",
+                  fn);
+    REQUIRE_PTR(a->k_cache, "k_cache");
+    REQUIRE_PTR(a->v_cache, "v_cache");
+    REQUIRE_PTR(a->block_table, "block_table");
+    REQUIRE_PTR(a->cache_lens, "cache_lens");
+    if (a->max_pages <= 0 || a->num_pages <= 0)
+      return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages and num_pages must be > 0 for a paged cache", fn);
+    mode = kModePaged;
+  } else {
+    if (a->total_k == 0) return fail(MIMO_ERR_INVALID_ARG, "%s: total_k must be > 0 without a paged cache", fn);
+    REQUIRE_PTR(a->k, "k");
+    REQUIRE_PTR(a->v, "v");
+    REQUIRE_PTR(a->cu_seqlens_k, "cu_seqlens_k");
+    if (a->cache_kind == MIMO_CACHE_RING) {
+      if (a->layer.window < 1 || a->layer.window > 129)
+        return fail(MIMO_ERR_INVALID_ARG, "%s: a ring cache needs a window of 1..129 keys", fn);
+      REQUIRE_PTR(a->k_cache, "k_cache");
+      REQUIRE_PTR(a->v_cache, "v_cache");
+      REQUIRE_PTR(a->cache_lens, "cache_lens");
+      mode = kModeExt;
+    } else {
+      mode = kModeContig;
+    }
+  }
+  const size_t need = mimo_attn_prefill_workspace_size(a->num_seqs, a->total_k, hkv, a->cache_kind);
+  if (need > 0) {
+    if (!a->workspace || a->workspace_bytes < need)
+      return fail(MIMO_ERR_WORKSPACE, "%s: workspace of %zu bytes required (got %zu)", fn, need,
+                  a->workspace ? a->workspace_bytes : size_t(0));
+    if (!aligned16(a->workspace)) return fail(MIMO_ERR_INVALID_ARG, "%s: workspace is not 16-byte aligned", fn);
+  }
+  const int kind = (a->layer.window >= 1 && a->layer.window <= 129 && mode != kModePaged) ? 0 : 1;
+  DevState d;
+  if (int rc = dev_state(fn, &d)) return rc;
+  EncodeTiledFn enc;
+  if (int rc = get_encoder(fn, &enc)) return rc;
+  const int tile_h = kind == 0 ? 8 : 16;  // query heads stacked in one M tile (one KV group)
+  if (kind == 0 && hkv != 8) return fail(MIMO_ERR_UNSUPPORTED, "%s: sliding-window path needs 8 KV heads", fn);
+  if (kind == 1 && hkv != 4) return fail(MIMO_ERR_UNSUPPORTED, "%s: global path needs 4 KV heads", fn);
+  const int R = prefill_rows_per_tile(kind);
+  const int BN = prefill_key_tile(kind);
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  int rc = make_map(fn, enc, &p.tm_q, a->q, a->total_q, kHq, kDqk, tile_h, R);
+  if (rc) return rc;
+  uint16_t* ws_k = static_cast<uint16_t*>(a->workspace);
+  uint16_t* ws_v = nullptr;
+  if (mode == kModeContig) {
+    if ((rc = make_map(fn, enc, &p.tm_k0, ws_k, a->total_k, hkv, kRope, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_k12, a->k, a->total_k, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_v, a->v, a->total_k, hkv, kDv, 1, BN))) return rc;
+  } else if (mode == kModeExt) {
+    const long rows = long(a->total_k) + 128L * a->num_seqs;
+    ws_v = reinterpret_cast<uint16_t*>(static_cast<char*>(a->workspace) + round256(size_t(rows) * hkv * kDqk * 2));
+    if ((rc = make_map(fn, enc, &p.tm_k0, ws_k, rows, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_k12, ws_k, rows, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_v, ws_v, rows, hkv, kDv, 1, BN))) return rc;
+  } else {
+    const long rows = long(a->num_pages) * kPage;
+    if ((rc = make_map(fn, enc, &p.tm_k0, a->k_cache, rows, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_k12, a->k_cache, rows, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, hkv, kDv, 1, BN))) return rc;
+  }
+  p.num_seqs = a->num_seqs;
+  p.total_q = a->total_q;
+  p.hkv = hkv;
+  p.mode = mode;
+  p.window = a->layer.window;
+  p.cu_q = a->cu_seqlens_q;
+  p.cu_k = a->cu_seqlens_k;
+  p.cache_lens = a->cache_lens;
+  p.block_table = a->block_table;
+  p.max_pages = a->max_pages;
+  p.num_pages = a->num_pages;
+  p.scale_log2 = a->layer.softmax_scale * 1.4426950408889634f;
+  p.v_scale = a->layer.v_scale;
+  p.sink = a->layer.sink;
+  p.out = static_cast<uint16_t*>(a->out);
+  p.lse = a->lse;
+  p.rope = make_freqs(a->layer.rope_base);
+  p.status = d.status;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode != kModePaged) {
+    RopeKParams r;
+    r.num_seqs = a->num_seqs;
+    r.total_k = a->total_k;
+    r.hkv = hkv;
+    r.mode = mode;
+    r.cu_k = a->cu_seqlens_k;
+    r.cache_lens = a->cache_lens;
+    r.k = static_cast<const uint16_t*>(a->k);
+    r.v = static_cast<const uint16_t*>(a->v);
+    r.ring_k = static_cast<const uint16_t*>(a->k_cache);
+    r.ring_v = static_cast<const uint16_t*>(a->v_cache);
+    r.ws_k = ws_k;
+    r.ws_v = ws_v;
+    r.rope = p.rope;
+    r.status = d.status;
+    cudaError_t e = launch_rope_k(r, st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: key pre-pass launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  // upper bound of M tiles: ceil(total_q / R) + num_seqs partial tiles, times KV heads
+  const long work = (long(a->total_q) / R + a->num_seqs + 1) * hkv;
+  const int grid = int(work < d.sms ? work : d.sms);
+  cudaError_t e = launch_prefill(p, kind, grid, st);
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return MIMO_OK;
+}
+
+int mimo_status_poll(uint32_t* status) {
+  const char* fn = "mimo_status_poll";
+  if (!status) return fail(MIMO_ERR_INVALID_ARG, "%s: status is NULL", fn);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v));
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  *status = v;
+  if (v & MIMO_STATUS_TIMEOUT) return fail(MIMO_ERR_TIMEOUT, "%s: a device wait gave up (status 0x%x)", fn, v);
+  return MIMO_OK;
+}
+
+}  // extern "C"

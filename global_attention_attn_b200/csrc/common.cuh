@@ -1,0 +1,49 @@
+// Device helpers shared by the kernels: bf16 conversion and the RoPE angle.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace mimo {
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  return uint32_t(f32_to_bf16(lo)) | (uint32_t(f32_to_bf16(hi)) << 16);
+}
+
+// cos / sin of pos * inv_freq.  The angle and its reduction to [-pi, pi] are
+// taken in float64 (the fastest rotary angle equals the position, up to ~1.3e5
+// radians here, far past where a float32 angle keeps its digits); only the
+// reduced angle goes through the float32 sincos.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double theta = double(pos) * inv_freq;
+  const double k = rint(theta * (1.0 / two_pi));
+  const float r = float(fma(-k, two_pi, theta));
+  sincosf(r, s, c);
+}
+
+// NeoX rotate-half on one 16-byte chunk pair: lo holds dims 8u..8u+7, hi holds
+// dims 8u+32..8u+39 (u in 0..3); frequency index of element i is 8u+i.
+__device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int pos, const RopeFreqs& rf) {
+  uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float x0 = lo_bf16(a[w]), x1 = hi_bf16(a[w]);
+    float y0 = lo_bf16(b[w]), y1 = hi_bf16(b[w]);
+    float c0, s0, c1, s1;
+    rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w], &c0, &s0);
+    rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w + 1], &c1, &s1);
+    a[w] = pack2_bf16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+    b[w] = pack2_bf16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1);
+  }
+}
+
+}  // namespace mimo

@@ -1,0 +1,110 @@
+// Internal launch interfaces shared by the host API (api.cu) and the kernel
+// translation units.  Not part of the public C ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace mimo {
+
+constexpr int kHq = 64;
+constexpr int kDqk = 192;
+constexpr int kDv = 128;
+constexpr int kRope = 64;
+constexpr int kHalf = kRope / 2;
+constexpr int kPage = 128;  // positions per page / ring slots
+
+// Rotary frequencies base^(-2j/64), j = 0..31, evaluated on the host in float64.
+struct RopeFreqs {
+  double inv_freq[kHalf];
+};
+
+struct AppendParams {
+  int num_tokens, hkv;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const int32_t* pos;
+  const int32_t* seq_idx;
+  int cache_kind;
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  int num_seqs;
+  const int32_t* block_table;
+  int max_pages, num_pages;
+  RopeFreqs rope;
+  unsigned* status;
+};
+
+struct DecodeParams {
+  int batch, hkv, group;  // group = 64 / hkv
+  int window;
+  int split_len, max_splits;
+  float scale_log2;  // softmax_scale * log2(e)
+  float v_scale;
+  const float* sink;
+  const uint16_t* q;
+  const int32_t* seq_lens;
+  int cache_kind;
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  const int32_t* block_table;
+  int max_pages, num_pages;
+  uint16_t* out;
+  float* lse;
+  float* ws_o;   // [batch, 64, max_splits, 128]
+  float* ws_ml;  // [batch, 64, max_splits, 2]
+  RopeFreqs rope;
+  unsigned* status;
+};
+
+// Key source modes of the prefill kernel.
+enum PrefillMode : int {
+  kModeContig = 0,  // dims 0..63 from the rotated workspace copy, 64..191 from k, v from v
+  kModeExt = 1,     // everything from the workspace copy [ring halo | new keys]
+  kModePaged = 2,   // everything from the paged cache
+};
+
+struct PrefillParams {
+  CUtensorMap tm_q;    // q [total_q, 64, 192], box {64, G, 128/G}
+  CUtensorMap tm_k0;   // key dims 0..63 source, box {64, 1, BN}
+  CUtensorMap tm_k12;  // key dims 64..191 source (x = 64, 128), box {64, 1, BN}
+  CUtensorMap tm_v;    // value source (x = 0, 64), box {64, 1, BN}
+  int num_seqs, total_q, hkv, mode, window;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const int32_t* cache_lens;
+  const int32_t* block_table;
+  int max_pages, num_pages;
+  float scale_log2;
+  float v_scale;
+  const float* sink;
+  uint16_t* out;
+  float* lse;
+  RopeFreqs rope;
+  unsigned* status;
+};
+
+// Pre-pass of the prefill: rotated key copies into the workspace.
+struct RopeKParams {
+  int num_seqs, total_k, hkv, mode;
+  const int32_t* cu_k;
+  const int32_t* cache_lens;
+  const uint16_t* k;
+  const uint16_t* v;
+  const uint16_t* ring_k;  // ext mode
+  const uint16_t* ring_v;
+  uint16_t* ws_k;  // contig: [total_k, hkv, 64]; ext: [total_k + 128*B, hkv, 192]
+  uint16_t* ws_v;  // ext: [total_k + 128*B, hkv, 128]
+  RopeFreqs rope;
+  unsigned* status;
+};
+
+cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s);
+// kind 0: sliding window (G=8 heads x 16 rows, one 144-key tile); kind 1: global (G=16 x 8 rows, 128-key tiles)
+cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s);
+int prefill_rows_per_tile(int kind);
+int prefill_key_tile(int kind);
+
+}  // namespace mimo

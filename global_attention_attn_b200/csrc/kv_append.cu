@@ -1,0 +1,63 @@
+// KV append: rotate the first 64 dims of each new key at its position and
+// store key and value into the ring or paged cache.
+//
+// Cache layout follows the serving pages: window-sized KV for the sliding
+// layers (gaudi-cookbook "MiMo-V2.6-Flash-RL", "Launch": window-sized KV for
+// the 39 sliding layers) kept here as a 128-slot ring per sequence, and paged
+// KV with block size 128 for the global layers (same page, "--block-size 128").
+#include "common.cuh"
+#include "../../include/mimoattn.h"
+
+namespace mimo {
+
+// One warp per (token, kv head).  Lanes 0..3 rotate the chunk pairs (u, u+4) of
+// dims 0..63; lanes 8..23 copy chunks 8..23 (dims 64..191); lanes 0..15 copy V.
+__global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
+  const int warp = int((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= p.num_tokens * p.hkv) return;
+  const int t = warp / p.hkv, g = warp % p.hkv;
+  const int pos = p.pos[t], s = p.seq_idx[t];
+  long entry;
+  if (s < 0 || s >= p.num_seqs || pos < 0) {
+    if (lane == 0) atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
+    return;
+  }
+  if (p.cache_kind == MIMO_CACHE_RING) {
+    entry = long(s) * kPage + (pos % kPage);
+  } else {
+    const int pi = pos / kPage;
+    const int page = pi < p.max_pages ? p.block_table[long(s) * p.max_pages + pi] : -1;
+    if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
+      return;
+    }
+    entry = long(page) * kPage + (pos % kPage);
+  }
+  const uint4* ks = reinterpret_cast<const uint4*>(p.k_new + (long(t) * p.hkv + g) * kDqk);
+  uint4* kd = reinterpret_cast<uint4*>(p.k_cache + (entry * p.hkv + g) * kDqk);
+  if (lane < 4) {
+    uint4 lo = __ldg(ks + lane), hi = __ldg(ks + lane + 4);
+    rope_chunk_pair(lo, hi, lane, pos, p.rope);
+    kd[lane] = lo;
+    kd[lane + 4] = hi;
+  } else if (lane >= 8 && lane < 24) {
+    kd[lane] = __ldg(ks + lane);
+  }
+  if (lane < 16) {
+    const uint4* vs = reinterpret_cast<const uint4*>(p.v_new + (long(t) * p.hkv + g) * kDv);
+    uint4* vd = reinterpret_cast<uint4*>(p.v_cache + (entry * p.hkv + g) * kDv);
+    vd[lane] = __ldg(vs + lane);
+  }
+}
+
+cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s) {
+  const long warps = long(p.num_tokens) * p.hkv;
+  if (warps == 0) return cudaSuccess;
+  const int block = 256;
+  const long grid = (warps * 32 + block - 1) / block;
+  kv_append_kernel<<<unsigned(grid), block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mimo

@@ -1,0 +1,213 @@
+/*
+ * libmimoattn — MiMo-V2.6-Flash hybrid attention forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the attention layer that the model pages state
+ * (radixark miles docs "MiMo-V2.6-Flash", section 1 "Key highlights" and
+ * section 5.4 "Notable quirks"; "Model techniques map" page, sections
+ * "Grouped-query attention", "Sliding-window attention", "Learnable attention
+ * sink", "Partial RoPE"; gaudi-cookbook "MiMo-V2.6-Flash-RL", "Required fixes"):
+ *
+ *   64 query heads, KV heads 8 (sliding-window layers) or 4 (global layers);
+ *   query head h reads KV head h / (64 / num_kv_heads);
+ *   Q/K head dim 192, V head dim 128; NeoX rotate-half RoPE on dims 0..63 with
+ *   frequencies base^(-2j/64), j = 0..31, angles taken from float64;
+ *   query at position p sees keys t with t <= p and (window == 0 or p - t < window);
+ *   z_t = softmax_scale * q.k_t; an optional per-query-head sink logit s_h joins
+ *   the softmax denominator and carries no value;
+ *   out = v_scale * sum_t softmax(z, s_h)_t v_t;   lse = ln(sum_t e^{z_t} + e^{s_h}).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, dense and row-major in the stated shape.  bf16 tensors are
+ *     passed as `void*` (IEEE bfloat16 bit patterns).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only
+ *     enqueue work: no host synchronisation, no memory allocation.
+ *   - Return MIMO_OK or a MIMO_ERR_* code; mimo_last_error() gives a message
+ *     (thread-local).  Arguments are validated on the host before any launch; a
+ *     rejected call enqueues nothing.
+ *   - Device-side problems (a bounded wait that ran out, an index outside a
+ *     cache) set bits in a device status word instead of faulting; read and
+ *     clear it with mimo_status_poll().
+ *   - The fixed model dimensions (64 / 192 / 128 / 64) are the only ones
+ *     supported; other values return MIMO_ERR_UNSUPPORTED.
+ */
+#ifndef MIMOATTN_H
+#define MIMOATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MIMO_API __attribute__((visibility("default")))
+#else
+#define MIMO_API
+#endif
+
+#define MIMO_OK 0
+#define MIMO_ERR_INVALID_ARG 1 /* a NULL / misaligned pointer, a bad size */
+#define MIMO_ERR_UNSUPPORTED 2 /* dims or head counts other than the model's */
+#define MIMO_ERR_WORKSPACE 3   /* workspace missing or smaller than required */
+#define MIMO_ERR_CUDA 4        /* a CUDA runtime / driver call failed */
+#define MIMO_ERR_TIMEOUT 5     /* a device wait gave up (from mimo_status_poll) */
+
+/* Device status bits reported by mimo_status_poll(). */
+#define MIMO_STATUS_TIMEOUT 1u    /* a bounded barrier / copy wait ran out */
+#define MIMO_STATUS_BAD_INDEX 2u  /* a page id, slot or position outside its cache */
+
+/* The attention layer.  num_q_heads 64, head_dim_qk 192, head_dim_v 128 and
+ * rope_dim 64 are required; num_kv_heads is 8 or 4. */
+typedef struct {
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim_qk;
+  int head_dim_v;
+  int rope_dim;
+  double rope_base;    /* 1e4 (sliding-window layers) or 1e7 (global layers); > 0 */
+  float softmax_scale; /* 1/sqrt(192) in the model */
+  float v_scale;       /* 0.707 in the model; applied to the output (attention is linear in V) */
+  int window;          /* keys in total including the query itself (128 in the model);
+                          0 = global causal attention */
+  const float* sink;   /* device fp32 [num_q_heads] sink logits, or NULL for no sink */
+} mimo_layer;
+
+#define MIMO_CACHE_NONE 0
+#define MIMO_CACHE_PAGED 1 /* [num_pages, 128, Hkv, D] pages of 128 positions, via block_table */
+#define MIMO_CACHE_RING 2  /* [num_seqs, 128, Hkv, D]: position p of sequence s in slot p % 128 */
+
+/*
+ * Prefill (varlen, causal, window or global, sink on/off).
+ *
+ * Sequence s has q_len = cu_seqlens_q[s+1]-cu_seqlens_q[s] query rows and
+ * k_len = cu_seqlens_k[s+1]-cu_seqlens_k[s] new (pre-RoPE) key/value rows.
+ * Its context length is ctx = cache_lens[s] + k_len (cache_lens NULL = 0).
+ * Queries sit at positions ctx - q_len .. ctx - 1 (bottom-right aligned), new
+ * keys at positions cache_lens[s] .. ctx - 1, and positions below cache_lens[s]
+ * are read from the cache, where keys are stored already rotated.
+ *
+ *   MIMO_CACHE_NONE : all keys are new; k, v, cu_seqlens_k required.
+ *   MIMO_CACHE_RING : sliding-window chunk: the ring holds the positions
+ *                     cache_lens[s]-128 .. cache_lens[s]-1 (the prefix tail, not yet
+ *                     overwritten by this chunk); requires window in 1..129.
+ *   MIMO_CACHE_PAGED: all keys come from the paged cache (append the chunk with
+ *                     mimo_kv_append first); k, v, cu_seqlens_k must be NULL and
+ *                     cache_lens[s] is the full context length.
+ *
+ * Layouts: q [total_q, 64, 192] bf16 pre-RoPE; k [total_k, Hkv, 192] bf16
+ * pre-RoPE; v [total_k, Hkv, 128] bf16; out [total_q, 64, 128] bf16;
+ * lse [total_q, 64] fp32 natural-log LSE including the sink (may be NULL).
+ * The workspace (size from mimo_attn_prefill_workspace_size) holds rotated
+ * key copies; its contents need no initialisation.
+ * Cache slots at or beyond a sequence's context must hold finite values
+ * (e.g. zero-initialise caches): they are read and masked, not skipped.
+ */
+typedef struct {
+  mimo_layer layer;
+  int num_seqs;
+  int total_q;
+  int total_k;              /* rows of k / v (0 for MIMO_CACHE_PAGED) */
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu_seqlens_q; /* device int32 [num_seqs+1] */
+  const int32_t* cu_seqlens_k; /* device int32 [num_seqs+1] or NULL (paged) */
+  const int32_t* cache_lens;   /* device int32 [num_seqs] or NULL */
+  int cache_kind;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table; /* paged: device int32 [num_seqs, max_pages] */
+  int max_pages;
+  int num_pages; /* paged: pages in the pool */
+  void* out;
+  float* lse;
+  void* workspace;
+  size_t workspace_bytes;
+} mimo_prefill_args;
+
+/* Bytes of workspace mimo_attn_prefill needs for these sizes. */
+MIMO_API size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_k, int num_kv_heads, int cache_kind);
+
+MIMO_API int mimo_attn_prefill(const mimo_prefill_args* args, void* stream);
+
+/*
+ * Decode: one query token per sequence.  Token s sits at position
+ * seq_lens[s] - 1 and the cache already holds positions 0 .. seq_lens[s]-1
+ * (append the token with mimo_kv_append first).  Sliding-window layers use a
+ * ring cache (only the last 128 positions are kept); global layers a paged cache.
+ *
+ * Layouts: q [batch, 64, 192] bf16 pre-RoPE; out [batch, 64, 128] bf16;
+ * lse [batch, 64] fp32 or NULL.  max_seq_len is a host-side upper bound of
+ * seq_lens (it sizes the split-KV grid and the workspace).
+ */
+typedef struct {
+  mimo_layer layer;
+  int batch;
+  int max_seq_len;
+  const void* q;
+  const int32_t* seq_lens; /* device int32 [batch], each >= 1 */
+  int cache_kind;          /* MIMO_CACHE_PAGED or MIMO_CACHE_RING */
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table; /* paged: device int32 [batch, max_pages] */
+  int max_pages;
+  int num_pages;
+  void* out;
+  float* lse;
+  void* workspace;
+  size_t workspace_bytes;
+} mimo_decode_args;
+
+/* Bytes of workspace mimo_attn_decode needs (split-KV partials). */
+MIMO_API size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int num_kv_heads, int window);
+
+MIMO_API int mimo_attn_decode(const mimo_decode_args* args, void* stream);
+
+/*
+ * KV append: rotates the first 64 dims of each new key at its position (the
+ * layer's RoPE base, angles from float64) and stores key and value (value
+ * unscaled) in the cache: ring slot pos % 128 of sequence seq_idx[t], or page
+ * block_table[seq_idx[t]][pos / 128], slot pos % 128.
+ *
+ * Layouts: k_new [num_tokens, Hkv, 192] bf16 pre-RoPE; v_new [num_tokens, Hkv, 128];
+ * pos, seq_idx: device int32 [num_tokens].  Two tokens must not target the same slot.
+ */
+typedef struct {
+  int num_tokens;
+  int num_kv_heads;
+  int head_dim_qk;
+  int head_dim_v;
+  int rope_dim;
+  double rope_base;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* pos;
+  const int32_t* seq_idx;
+  int cache_kind;
+  void* k_cache;
+  void* v_cache;
+  int num_seqs;               /* ring: sequences in the ring cache */
+  const int32_t* block_table; /* paged: device int32 [num_seqs, max_pages] */
+  int max_pages;
+  int num_pages;
+} mimo_append_args;
+
+MIMO_API int mimo_kv_append(const mimo_append_args* args, void* stream);
+
+/* Thread-local message for the last error returned on this thread. */
+MIMO_API const char* mimo_last_error(void);
+
+/* Reads and clears the device status word of the current device
+ * (synchronises the device).  Returns MIMO_STATUS_* bits in *status. */
+MIMO_API int mimo_status_poll(uint32_t* status);
+
+/* Library version string. */
+MIMO_API const char* mimo_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMOATTN_H */

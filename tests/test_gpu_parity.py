@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle, element by
+element, on the same seeded inputs.
+
+Bar (bf16 output, fp32 accumulation): max-abs 2e-2 and mean-abs 2e-3 on O, 1e-3
+on the LSE.  Small cases are checked on every row; the full-size workloads on
+sampled rows (the oracle evaluates rows one by one), always including the rows
+at the window edge (126, 127, 128), the first and the last.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import configs, synth
+
+from .util import (chunked_cfg, decode_cfg, dev_bf16, dev_f32, dev_i32, host_f64, parity, prefill_cfg)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    import global_attention_attn_b200 as M
+    M.lib()
+    yield
+    assert M.status_poll() == 0, "device status word reported a timeout or a bad index"
+
+
+def make_prefill(lens, hkv, base, window, sink, seed, klens=None):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    klens = lens if klens is None else klens
+    cuk = np.concatenate([[0], np.cumsum(klens)]).astype(np.int32)
+    q = configs.bf16_normal(seed, 1, (int(cu[-1]), 64, 192))
+    k = configs.bf16_normal(seed, 2, (int(cuk[-1]), hkv, 192))
+    v = configs.bf16_normal(seed, 3, (int(cuk[-1]), hkv, 128))
+    s = synth.normal_f32(synth.stream_seed(seed, 4), (64,)) if sink else None
+    return configs.Prefill(configs.Layer("swa" if window else "global", hkv, base, window, s), q, k, v, cu, cuk)
+
+
+def check_prefill(cfg, rows=None, what=""):
+    out, lse = prefill_cfg(cfg)
+    ro, rl = oracle.prefill(cfg, rows=rows)
+    if rows is not None:
+        import torch
+        idx = torch.as_tensor(np.asarray(rows), dtype=torch.long, device=out.device)
+        out, lse = out[idx], lse[idx]
+    return parity(out, lse, ro, rl, what)
+
+
+# ----------------------------------------------------------------------------- KV append
+
+@pytest.mark.parametrize("kind", ["ring", "paged"])
+def test_kv_append(kind):
+    import torch
+    import global_attention_attn_b200 as M
+    n, hkv, base = 700, (8 if kind == "ring" else 4), (1e4 if kind == "ring" else 1e7)
+    k = configs.bf16_normal(41, 1, (n, hkv, 192))
+    v = configs.bf16_normal(41, 2, (n, hkv, 128))
+    seq = (np.arange(n) % 3).astype(np.int32)
+    pos = (np.arange(n) // 3 + np.array([0, 5, 120000])[seq]).astype(np.int32)
+    if kind == "ring":
+        kc = torch.zeros((3, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros((3, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
+        M.mimo_kv_append(dev_bf16(k), dev_bf16(v), dev_i32(pos), dev_i32(seq), rope_base=base,
+                         cache_kind=M.MIMO_CACHE_RING, k_cache=kc, v_cache=vc, num_seqs=3)
+        where = {(int(seq[t]), int(pos[t] % 128)): t for t in range(n)}   # last writer of each slot
+        slot = lambda s, sl: (s, sl)  # noqa: E731
+    else:
+        maxp = (int(pos.max()) // 128) + 1
+        bt = (synth.permutation(7, 3 * maxp).reshape(3, maxp)).astype(np.int32)
+        kc = torch.zeros((3 * maxp, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros((3 * maxp, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
+        M.mimo_kv_append(dev_bf16(k), dev_bf16(v), dev_i32(pos), dev_i32(seq), rope_base=base,
+                         cache_kind=M.MIMO_CACHE_PAGED, k_cache=kc, v_cache=vc, num_seqs=3,
+                         block_table=dev_i32(bt), num_pages=3 * maxp)
+        where = {(int(bt[seq[t], pos[t] // 128]), int(pos[t] % 128)): t for t in range(n)}
+    ko, vo = oracle.kv_append(k, v, pos, base)
+    kcn, vcn = host_f64(kc), host_f64(vc)
+    touched = np.zeros(kcn.shape[:2], bool)
+    for (a, b), t in where.items():
+        touched[a, b] = True
+        # rotated dims: fp32 rotation of bf16 inputs, rounded to bf16
+        assert np.all(np.abs(kcn[a, b, :, :64] - ko[t, :, :64]) <= 2.0 ** -8 * np.abs(ko[t, :, :64]) + 1e-5)
+        np.testing.assert_array_equal(kcn[a, b, :, 64:], ko[t, :, 64:])     # pass-through dims: exact
+        np.testing.assert_array_equal(vcn[a, b], vo[t])                       # values: exact copy
+    assert np.all(kcn[~touched] == 0) and np.all(vcn[~touched] == 0)
+
+
+# ----------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("ctx_range", [(1, 127), (100, 3000), (4096, 9000)])
+def test_decode_small(ctx_range):
+    sw, gl = configs.config3(seed=100 + ctx_range[0], B=8, ctx_range=ctx_range)
+    for cfg in (sw, gl):
+        out, lse = decode_cfg(cfg)
+        ro, rl = oracle.decode(cfg)
+        parity(out, lse, ro, rl, cfg.name)
+
+
+def test_decode_split_boundaries():
+    # contexts on both sides of the 512-key split length and of one page
+    import global_attention_attn_b200 as M
+    sw, gl = configs.config3(seed=321, B=8, ctx_range=(1, 2))
+    ctx = np.array([1, 127, 128, 129, 511, 512, 513, 1025], np.int32)
+    bt, pool = configs.paged_layout(5, 1, ctx)
+    gl = configs.Decode(gl.layer, gl.q, ctx, configs.bf16_normal(5, 2, (pool, 128, 4, 192)),
+                        configs.bf16_normal(5, 3, (pool, 128, 4, 128)), block_table=bt)
+    out, lse = decode_cfg(gl)
+    ro, rl = oracle.decode(gl)
+    parity(out, lse, ro, rl, "global split boundaries")
+    sw = configs.Decode(sw.layer, sw.q, ctx, sw.k_cache, sw.v_cache)
+    out, lse = decode_cfg(sw)
+    ro, rl = oracle.decode(sw)
+    parity(out, lse, ro, rl, "swa ring wrap")
+    assert M.status_poll() == 0
+
+
+@pytest.fixture(scope="module")
+def cfg3():
+    return configs.config3()
+
+
+def test_decode_config3_swa_ring(cfg3):
+    sw, _ = cfg3
+    out, lse = decode_cfg(sw)
+    ro, rl = oracle.decode(sw)
+    parity(out, lse, ro, rl, "config 3 swa ring, all 64 sequences")
+
+
+def test_decode_config3_global_paged(cfg3):
+    _, gl = cfg3
+    out, lse = decode_cfg(gl)
+    seqs = np.array(sorted(set([0, 63] + list(synth.permutation(77, 64)[:6]))))
+    ro, rl = oracle.decode(gl, seqs=seqs)
+    import torch
+    idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "config 3 global paged, sampled sequences")
+
+
+# ----------------------------------------------------------------------------- prefill: sliding window
+
+def test_prefill_config0():
+    check_prefill(configs.config0(), what="config 0")
+
+
+@pytest.mark.parametrize("lens", [[1], [16], [127, 128, 129], [1, 15, 16, 17, 31, 300], [1000]])
+def test_prefill_swa_edges(lens):
+    check_prefill(make_prefill(lens, 8, 1e4, 128, True, 200 + sum(lens)), what=f"swa {lens}")
+
+
+def test_prefill_swa_no_sink():
+    check_prefill(make_prefill([513, 77], 8, 1e4, 128, False, 301), what="swa no sink")
+
+
+def test_prefill_swa_window_129():
+    # the SGLang / miles window convention: the query plus 128 previous keys
+    check_prefill(make_prefill([400], 8, 1e4, 129, True, 302), what="swa window 129")
+
+
+def test_prefill_swa_small_window():
+    check_prefill(make_prefill([300], 8, 1e4, 5, True, 303), what="swa window 5")
+
+
+def test_prefill_swa_fewer_queries_than_keys():
+    # bottom-right alignment: 40 queries at the end of 300 keys
+    check_prefill(make_prefill([40], 8, 1e4, 128, True, 304, klens=[300]), what="swa q<k")
+
+
+def test_prefill_config1_sampled():
+    cfg = configs.config1()
+    cu = cfg.cu_q
+    always = set()
+    for s in range(cfg.num_seqs):
+        for r in (0, 1, 15, 16, 126, 127, 128, 129):
+            always.add(int(cu[s] + r))
+        always.add(int(cu[s + 1] - 1))
+    rows = configs.sample_rows(11, int(cu[-1]), 1024, always=sorted(always))
+    check_prefill(cfg, rows=rows, what="config 1 (sampled rows)")
+
+
+# ----------------------------------------------------------------------------- prefill: global
+
+@pytest.mark.parametrize("lens", [[1], [8, 9], [1, 127, 128, 129, 300], [1500]])
+def test_prefill_global_small(lens):
+    check_prefill(make_prefill(lens, 4, 1e7, 0, False, 400 + sum(lens)), what=f"global {lens}")
+
+
+def test_prefill_global_with_sink_and_wide_window():
+    check_prefill(make_prefill([700], 4, 1e7, 300, True, 410), what="global window 300 + sink")
+
+
+def test_prefill_config2_sampled():
+    cfg = configs.config2()
+    rows = configs.sample_rows(22, 16384, 96, always=(0, 1, 7, 8, 127, 128, 129, 8191, 16383))
+    check_prefill(cfg, rows=rows, what="config 2 (sampled rows)")
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+
+def test_chunked_small_unaligned():
+    glb, swa = configs.config4(seed=55, prefix=1000, chunk=300, n_sample=300)
+    for cfg in (glb, swa):
+        out, lse = chunked_cfg(cfg)
+        ro, rl = oracle.chunked(cfg, rows=np.arange(300))
+        parity(out, lse, ro, rl, cfg.name)
+
+
+def test_chunked_config4():
+    glb, swa = configs.config4()
+    out, lse = chunked_cfg(swa)
+    ro, rl = oracle.chunked(swa)
+    import torch
+    idx = torch.as_tensor(swa.sample_rows, dtype=torch.long, device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "config 4 swa chunk (1024 sampled rows)")
+    out, lse = chunked_cfg(glb)
+    rows = configs.sample_rows(4, 8192, 48, always=(0, 126, 127, 128, 8191))
+    ro, rl = oracle.chunked(glb, rows=rows)
+    idx = torch.as_tensor(rows, dtype=torch.long, device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "config 4 global chunk (sampled rows)")
+
+
+# ----------------------------------------------------------------------------- cross-path
+
+def test_decode_matches_last_prefill_row():
+    """Appending a sequence to the caches and decoding its last token gives the last prefill row."""
+    import torch
+    import global_attention_attn_b200 as M
+    for hkv, base, window, sink in [(8, 1e4, 128, True), (4, 1e7, 0, False)]:
+        S = 700
+        cfg = make_prefill([S], hkv, base, window, sink, 500 + hkv)
+        out, lse = prefill_cfg(cfg)
+        pos = np.arange(S, dtype=np.int32)
+        seq = np.zeros(S, np.int32)
+        if window:
+            kc = torch.zeros((1, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
+            vc = torch.zeros((1, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
+            extra = dict(cache_kind=M.MIMO_CACHE_RING)
+        else:
+            npg = (S + 127) // 128
+            bt = dev_i32(synth.permutation(3, npg)[None, :])
+            kc = torch.zeros((npg, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
+            vc = torch.zeros((npg, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
+            extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=bt, num_pages=npg)
+        M.mimo_kv_append(dev_bf16(cfg.k), dev_bf16(cfg.v), dev_i32(pos), dev_i32(seq), rope_base=base,
+                         k_cache=kc, v_cache=vc, num_seqs=1, **extra)
+        dout, dlse = M.mimo_attn_decode(dev_bf16(cfg.q[S - 1:]), dev_i32([S]), max_seq_len=S, num_kv_heads=hkv,
+                                        rope_base=base, window=window, sink=dev_f32(cfg.layer.sink), k_cache=kc,
+                                        v_cache=vc, **extra)
+        d = (dout.float() - out[S - 1:].float()).abs()
+        assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3
+        assert (dlse - lse[S - 1:]).abs().max().item() <= 1e-3
