@@ -1,0 +1,552 @@
+#!/usr/bin/env python
+"""Benchmark of the MiMo-V2.6-Flash hybrid attention forward (libmimoattn) on B200.
+
+A step is one pass of the hot path over one batch: the sliding-window layer's
+varlen prefill of 8 sequences with lengths uniform in [1024, 8192] (RoPE on Q/K,
+QK^T, window-128 mask, online softmax with the per-head sink, PV, epilogue).
+`value` is algorithmic TFLOP/s (640 FLOP per visible (query head, key) pair)
+over all GPUs; each GPU runs its own replica of the workload (the path has no
+exchange step: "weak" scaling, replicas only).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--main-only]
+
+With --gpus N > 1 launch it under torchrun (one process per GPU).  Rank 0
+prints one JSON line.  Besides the contract keys the line carries `per_config`:
+the other four workloads measured the same way (prefill TFLOP/s, decode GB/s,
+fraction of the roofline max(FLOP / bf16 peak, bytes / HBM peak)).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import configs  # noqa: E402
+
+METRIC = "SWA+sink / global attn prefill TFLOP/s, decode KV GB/s; % of B200 roofline"
+FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) pair
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel, from the ncu
+# capture summarised in profiles/ (None until a capture of the current kernel exists).
+TRAFFIC_BYTES = {"prefill_kernel<0>/swa_varlen_prefill": None}
+
+
+# ----------------------------------------------------------------------------- roofline inputs
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def prefill_counts(cfg):
+    """Algorithmic FLOP and bytes of a contiguous prefill (workloads.configs.Prefill)."""
+    pairs = 0
+    for s in range(cfg.num_seqs):
+        ql, kl = int(cfg.q_lens[s]), int(cfg.k_lens[s])
+        pos = np.arange(kl - ql, kl, dtype=np.int64)
+        vis = np.minimum(pos + 1, cfg.layer.window) if cfg.layer.window else pos + 1
+        pairs += int(vis.sum())
+    tq, tk, h = int(cfg.cu_q[-1]), int(cfg.cu_k[-1]), cfg.layer.num_kv_heads
+    by = tq * 64 * (192 * 2 + 128 * 2 + 4) + tk * h * (192 + 128) * 2 + 4 * (2 * cfg.num_seqs + 2)
+    return pairs * 64 * FLOP_PER_PAIR, by
+
+
+def decode_counts(cfg):
+    L = cfg.layer
+    vis = np.minimum(cfg.ctx, L.window) if L.window else cfg.ctx
+    keys = int(vis.astype(np.int64).sum())
+    B = len(cfg.ctx)
+    by = keys * L.num_kv_heads * (192 + 128) * 2 + B * 64 * (192 * 2 + 128 * 2 + 4) + B * 4
+    if cfg.paged:
+        by += int(((cfg.ctx + 127) // 128).sum()) * 4
+    return keys * 64 * FLOP_PER_PAIR, by
+
+
+def chunked_counts(cfg):
+    L = cfg.layer
+    n = int(cfg.cu_new[-1])
+    start = int(cfg.start[0])
+    pos = start + np.arange(n, dtype=np.int64)
+    vis = np.minimum(pos + 1, L.window) if L.window else pos + 1
+    ctx = start + n
+    keys_read = (min(ctx, n + L.window - 1) if L.window else ctx)
+    by = n * 64 * (192 * 2 + 128 * 2 + 4) + keys_read * L.num_kv_heads * (192 + 128) * 2
+    if cfg.paged:
+        by += n * L.num_kv_heads * (192 + 128) * 2 * 2  # the append reads the chunk and writes it
+    return int(vis.sum()) * 64 * FLOP_PER_PAIR, by
+
+
+def roofline_us(flops, by, hbm, tf):
+    return max(flops / (tf * 1e12), by / (hbm * 1e9)) * 1e6
+
+
+# ----------------------------------------------------------------------------- clocks
+
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~10 ms."""
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it, never guess
+            self.h, self.err = None, f"nvml unavailable: {e}"
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_reasons(self.h)
+                for bit, name in _REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.h is not None:
+            self.t.join()
+
+    def summary(self):
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+             "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        if self.err:
+            d["note"] = self.err
+        return d
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dev_bf16(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_i32(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.int32))).cuda()
+
+
+def dev_f32(a):
+    import torch
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.float32))).cuda()
+
+
+def event_time_ms(fn, iters, flush=None):
+    """Device time of `iters` calls of fn on the current stream (CUDA events, synchronised on
+    both sides).  With `flush`, L2 is flushed before each call and only the calls are timed."""
+    import torch
+    s = torch.cuda.current_stream()
+    if flush is None:
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(iters):
+            fn()
+        b.record(s)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+    tot = 0.0
+    for _ in range(iters):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        torch.cuda.synchronize()
+        tot += a.elapsed_time(b)
+    return tot
+
+
+class Prefill:
+    """Device-resident prefill workload plus the call through the C ABI."""
+
+    def __init__(self, cfg):
+        import torch
+        import global_attention_attn_b200 as M
+        self.cfg, self.M = cfg, M
+        L = cfg.layer
+        self.q, self.k, self.v = dev_bf16(cfg.q), dev_bf16(cfg.k), dev_bf16(cfg.v)
+        self.cq, self.ck, self.sink = dev_i32(cfg.cu_q), dev_i32(cfg.cu_k), dev_f32(L.sink)
+        T = self.q.shape[0]
+        self.out = torch.empty((T, 64, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((T, 64), dtype=torch.float32, device="cuda")
+        n = M.prefill_workspace_size(cfg.num_seqs, self.k.shape[0], L.num_kv_heads, M.MIMO_CACHE_NONE)
+        self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        L = self.cfg.layer
+        self.M.mimo_attn_prefill(self.q, self.k, self.v, self.cq, self.ck, num_kv_heads=L.num_kv_heads,
+                                 rope_base=L.rope_base, window=L.window, sink=self.sink, out=self.out, lse=self.lse,
+                                 workspace=self.ws)
+
+
+class Decode:
+    def __init__(self, cfg):
+        import torch
+        import global_attention_attn_b200 as M
+        self.cfg, self.M = cfg, M
+        L = cfg.layer
+        self.q, self.ctx = dev_bf16(cfg.q), dev_i32(cfg.ctx)
+        self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
+        self.sink = dev_f32(L.sink)
+        self.extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
+                          num_pages=cfg.k_cache.shape[0]) if cfg.paged else dict(cache_kind=M.MIMO_CACHE_RING)
+        B = self.q.shape[0]
+        self.out = torch.empty((B, 64, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((B, 64), dtype=torch.float32, device="cuda")
+        n = M.decode_workspace_size(B, int(cfg.ctx.max()), L.num_kv_heads, L.window)
+        self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        L = self.cfg.layer
+        self.M.mimo_attn_decode(self.q, self.ctx, max_seq_len=int(self.cfg.ctx.max()), num_kv_heads=L.num_kv_heads,
+                                rope_base=L.rope_base, window=L.window, k_cache=self.kc, v_cache=self.vc,
+                                sink=self.sink, out=self.out, lse=self.lse, workspace=self.ws, **self.extra)
+
+
+class Chunked:
+    """Global layer: append the chunk to the paged cache, then prefill from the cache.
+    Sliding layer: prefill from the ring (prefix tail) plus the new rows."""
+
+    def __init__(self, cfg):
+        import torch
+        import global_attention_attn_b200 as M
+        self.cfg, self.M = cfg, M
+        L = cfg.layer
+        n = int(cfg.cu_new[-1])
+        self.q, self.k, self.v = dev_bf16(cfg.q), dev_bf16(cfg.k_new), dev_bf16(cfg.v_new)
+        self.cu = dev_i32(cfg.cu_new)
+        self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
+        self.sink = dev_f32(L.sink)
+        self.out = torch.empty((n, 64, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((n, 64), dtype=torch.float32, device="cuda")
+        if cfg.paged:
+            self.bt = dev_i32(cfg.block_table)
+            self.pos = dev_i32(cfg.start[0] + np.arange(n))
+            self.seq = dev_i32(np.zeros(n))
+            self.ctx = dev_i32(cfg.start + n)
+            self.ws = None
+        else:
+            self.start = dev_i32(cfg.start)
+            w = M.prefill_workspace_size(1, n, L.num_kv_heads, M.MIMO_CACHE_RING)
+            self.ws = torch.empty(w, dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        M, L, cfg = self.M, self.cfg.layer, self.cfg
+        if cfg.paged:
+            M.mimo_kv_append(self.k, self.v, self.pos, self.seq, rope_base=L.rope_base, cache_kind=M.MIMO_CACHE_PAGED,
+                             k_cache=self.kc, v_cache=self.vc, num_seqs=1, block_table=self.bt,
+                             num_pages=cfg.k_cache.shape[0])
+            M.mimo_attn_prefill(self.q, None, None, self.cu, None, num_kv_heads=L.num_kv_heads, rope_base=L.rope_base,
+                                window=L.window, sink=self.sink, cache_lens=self.ctx, cache_kind=M.MIMO_CACHE_PAGED,
+                                k_cache=self.kc, v_cache=self.vc, block_table=self.bt,
+                                num_pages=cfg.k_cache.shape[0], out=self.out, lse=self.lse)
+        else:
+            M.mimo_attn_prefill(self.q, self.k, self.v, self.cu, self.cu, num_kv_heads=L.num_kv_heads,
+                                rope_base=L.rope_base, window=L.window, sink=self.sink, cache_lens=self.start,
+                                cache_kind=M.MIMO_CACHE_RING, k_cache=self.kc, v_cache=self.vc, out=self.out,
+                                lse=self.lse, workspace=self.ws)
+
+
+def l2_flusher():
+    import torch
+    buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    return lambda: buf.fill_(1)
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+
+def cpu_baseline(cfg, max_seconds=12.0):
+    """The float64 oracle, as it stands, on a bounded sample of the workload's query rows."""
+    import oracle
+    cores = oracle.default_threads()
+    total = int(cfg.cu_q[-1])
+    # calibrate on a small sample, then size the sample to about max_seconds
+    probe = configs.sample_rows(7, total, 256)
+    t0 = time.perf_counter()
+    oracle.prefill(cfg, rows=probe, nthreads=cores)
+    dt = time.perf_counter() - t0
+    n = int(min(total, max(256, 256 * max_seconds / max(dt, 1e-3))))
+    rows = configs.sample_rows(8, total, n)
+    t0 = time.perf_counter()
+    oracle.prefill(cfg, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    flops = _rows_flops(cfg, rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} of {total} query rows (all 64 heads), float64, {dt:.1f} s"}
+
+
+def _rows_flops(cfg, rows):
+    cu = cfg.cu_q.astype(np.int64)
+    seq = np.searchsorted(cu, rows, side="right") - 1
+    pos = (cfg.q_pos0[seq] + (rows - cu[seq])).astype(np.int64)
+    vis = np.minimum(pos + 1, cfg.layer.window) if cfg.layer.window else pos + 1
+    return int(vis.sum()) * 64 * FLOP_PER_PAIR
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is a bounded sample of the same workload."""
+    if rank != 0:
+        return 0
+    import oracle
+    cfg = configs.config1()
+    cores = oracle.default_threads()
+    total = int(cfg.cu_q[-1])
+    # size each step's sample so that warmup + steps take about two minutes of CPU time
+    probe = configs.sample_rows(7, total, 256)
+    t0 = time.perf_counter()
+    oracle.prefill(cfg, rows=probe, nthreads=cores)
+    per_row = (time.perf_counter() - t0) / 256
+    n = int(min(4096, max(64, 120.0 / max(1, args.steps + args.warmup) / max(per_row, 1e-7))))
+    rows = configs.sample_rows(9, total, n)
+    flops = _rows_flops(cfg, rows)
+    for _ in range(args.warmup):
+        oracle.prefill(cfg, rows=rows, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.prefill(cfg, rows=rows, nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "num_seqs": cfg.num_seqs, "total_tokens": int(cfg.cu_q[-1]),
+                       "window": 128, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{len(rows)} of {int(cfg.cu_q[-1])} query rows per step (all 64 heads)"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--main-only", action="store_true", help="skip the per-config details and the CPU baseline")
+    ap.add_argument("--profile", choices=["swa", "global", "decode"],
+                    help="run only a small case of one kernel (inputs > L2, < 1 GB on the device) for ncu captures")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    import global_attention_attn_b200 as M
+    M.lib()
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    if args.profile:
+        return run_profile_case(args)
+
+    def barrier():
+        if pg:
+            pg.barrier()
+
+    # ---------------- the timed workload: sliding-window varlen prefill
+    cfg = configs.config1()
+    flops, by = prefill_counts(cfg)
+    step = Prefill(cfg)
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_ms = event_time_ms(step, args.steps)
+    barrier()
+    if pg:
+        t = torch.tensor([t_ms], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        t_ms = float(t.item())
+    ms_step = t_ms / args.steps
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    achieved = by / (ms_step * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": TRAFFIC_BYTES["prefill_kernel<0>/swa_varlen_prefill"],
+            "kernel": "prefill (key pre-pass + tcgen05 prefill_kernel<0>)", "peak_source": f"{peak_src} hbm_gbs",
+            "algorithmic_bytes": by, "algorithmic_flop": flops,
+            "tensor_frac": flops / (ms_step * 1e-3) / 1e12 / tf_sust}
+
+    # ---------------- end to end through the C ABI: host buffers, copies inside the timed region
+    q_h = step.q.cpu().pin_memory()
+    k_h, v_h = step.k.cpu().pin_memory(), step.v.cpu().pin_memory()
+    cq_h, ck_h = step.cq.cpu().pin_memory(), step.ck.cpu().pin_memory()
+    s_h = step.sink.cpu().pin_memory()
+    out_h, lse_h = torch.empty_like(step.out, device="cpu").pin_memory(), torch.empty_like(step.lse, device="cpu").pin_memory()
+
+    def e2e_step():
+        step.q.copy_(q_h, non_blocking=True)
+        step.k.copy_(k_h, non_blocking=True)
+        step.v.copy_(v_h, non_blocking=True)
+        step.cq.copy_(cq_h, non_blocking=True)
+        step.ck.copy_(ck_h, non_blocking=True)
+        step.sink.copy_(s_h, non_blocking=True)
+        step()
+        out_h.copy_(step.out, non_blocking=True)
+        lse_h.copy_(step.lse, non_blocking=True)
+
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, cq_h, ck_h, s_h))
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    for _ in range(2):
+        e2e_step()
+    ke = max(3, min(args.steps, 10))
+    barrier()
+    te = event_time_ms(e2e_step, ke) / ke
+    if pg:
+        t = torch.tensor([te], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        te = float(t.item())
+    e2e = {"value": flops * world / (te * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": te}
+    del q_h, k_h, v_h, out_h, lse_h
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "num_seqs": cfg.num_seqs, "total_tokens": int(cfg.cu_q[-1]),
+                       "q_heads": 64, "kv_heads": 8, "head_dim_qk": 192, "head_dim_v": 128, "window": 128,
+                       "sink": True, "rope_base": 1e4, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2 ({by / 1e9:.2f} GB moved per step)"},
+            "roofline": roof, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+
+    # ---------------- per-config details and the CPU baseline (rank 0, one GPU)
+    if rank == 0 and world == 1 and not args.main_only:
+        del step
+        torch.cuda.empty_cache()
+        per = {}
+        flush = l2_flusher()
+        c0 = configs.config0()
+        f0, b0 = prefill_counts(c0)
+        w0 = Prefill(c0)
+        for _ in range(3):
+            w0()
+        t0 = event_time_ms(w0, 50, flush=flush) / 50
+        per["swa_prefill_s512"] = _entry(f0, b0, t0, hbm, tf_burst, "L2 flushed before each call")
+        del w0
+        c2 = configs.config2()
+        f2, b2 = prefill_counts(c2)
+        w2 = Prefill(c2)
+        for _ in range(3):
+            w2()
+        t2 = event_time_ms(w2, 10) / 10
+        per["global_prefill_s16384"] = _entry(f2, b2, t2, hbm, tf_sust, "inputs larger than L2")
+        del w2, c2
+        torch.cuda.empty_cache()
+        sw, gl = configs.config3()
+        for name, c, fl in (("swa_decode_b64_ring128", sw, flush), ("global_decode_b64_paged128", gl, None)):
+            fd, bd = decode_counts(c)
+            w = Decode(c)
+            for _ in range(3):
+                w()
+            td = event_time_ms(w, 20, flush=fl) / 20
+            e = _entry(fd, bd, td, hbm, tf_burst, "L2 flushed before each call" if fl else "inputs larger than L2")
+            e["GB/s"] = bd / (td * 1e-3) / 1e9
+            per[name] = e
+            del w
+        del sw, gl
+        torch.cuda.empty_cache()
+        g4, s4 = configs.config4()
+        for name, c in (("global_chunk_8192_on_120832", g4), ("swa_chunk_8192_on_120832", s4)):
+            fc, bc = chunked_counts(c)
+            w = Chunked(c)
+            for _ in range(3):
+                w()
+            tc = event_time_ms(w, 5) / 5
+            per[name] = _entry(fc, bc, tc, hbm, tf_sust if c.paged else tf_burst, "inputs larger than L2")
+            del w
+        line["per_config"] = per
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    print(json.dumps(line), flush=True) if rank == 0 else None
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def profile_case(name):
+    """Small workloads of each kernel for profiler captures: inputs larger than L2 (126 MB),
+    well under a gigabyte on the device."""
+    if name == "swa":
+        lens = np.array([4096, 4096])
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        L = configs.swa_layer(configs.synth.normal_f32(configs.synth.stream_seed(5, 4), (64,)))
+        T = int(cu[-1])
+        return Prefill(configs.Prefill(L, configs.bf16_normal(5, 1, (T, 64, 192)), configs.bf16_normal(5, 2, (T, 8, 192)),
+                                       configs.bf16_normal(5, 3, (T, 8, 128)), cu, cu.copy(), name="swa_prefill_2x4096"))
+    if name == "global":
+        return Prefill(configs.config2(S=4096))
+    sw, gl = configs.config3(B=16)
+    return Decode(gl)
+
+
+def run_profile_case(args):
+    import torch
+    w = profile_case(args.profile)
+    for _ in range(args.warmup + args.steps):
+        w()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile, "launch_calls": args.warmup + args.steps}))
+    return 0
+
+
+def _entry(flops, by, ms, hbm, tf, l2):
+    troof = roofline_us(flops, by, hbm, tf)
+    return {"us": ms * 1e3, "TFLOP/s": flops / (ms * 1e-3) / 1e12, "GB/s": by / (ms * 1e-3) / 1e9,
+            "roofline_us": troof, "frac": troof / (ms * 1e3),
+            "bound": "tensor" if flops / (tf * 1e12) > by / (hbm * 1e9) else "hbm", "l2": l2}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

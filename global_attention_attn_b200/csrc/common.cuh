@@ -1,6 +1,7 @@
 // Device helpers shared by the kernels: bf16 conversion and the RoPE angle.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "internal.h"
@@ -15,6 +16,9 @@ __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return uint32_t(f32_to_bf16(lo)) | (uint32_t(f32_to_bf16(hi)) << 16);
+}
+__device__ __forceinline__ uint32_t pack2_f16(float lo, float hi) {
+  return uint32_t(__half_as_ushort(__float2half_rn(lo))) | (uint32_t(__half_as_ushort(__float2half_rn(hi))) << 16);
 }
 
 // cos / sin of pos * inv_freq.  The angle and its reduction to [-pi, pi] are
@@ -31,6 +35,9 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
 
 // NeoX rotate-half on one 16-byte chunk pair: lo holds dims 8u..8u+7, hi holds
 // dims 8u+32..8u+39 (u in 0..3); frequency index of element i is 8u+i.
+// Input bf16, output IEEE fp16: the rotated dims are kept in fp16 everywhere
+// (query tiles, key copies, caches) because their rounding error enters every
+// logit; fp16 has 11 significant bits against bf16's 8.
 __device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int pos, const RopeFreqs& rf) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
@@ -41,8 +48,8 @@ __device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int
     float c0, s0, c1, s1;
     rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w], &c0, &s0);
     rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w + 1], &c1, &s1);
-    a[w] = pack2_bf16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
-    b[w] = pack2_bf16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1);
+    a[w] = pack2_f16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+    b[w] = pack2_f16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1);
   }
 }
 

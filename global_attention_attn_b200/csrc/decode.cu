@@ -54,6 +54,14 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// fp16 operands: the rotated dims 0..63 (fp16 in the query tile and in the caches)
+__device__ __forceinline__ void mma16816_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -179,8 +187,13 @@ __global__ void __launch_bounds__(128, 2) decode_partial_kernel(const DecodePara
       for (int kk = 0; kk < 12; ++kk) {
         uint32_t b[4];
         ldsm_x4(smem_u32(kbuf + key * kKStride + (16 * kk + dof) * 2), b);
-        mma16816(acc0, qa[kk], b[0], b[1]);
-        mma16816(acc1, qa[kk], b[2], b[3]);
+        if (kk < 4) {  // dims 0..63: rotated, fp16
+          mma16816_f16(acc0, qa[kk], b[0], b[1]);
+          mma16816_f16(acc1, qa[kk], b[2], b[3]);
+        } else {
+          mma16816(acc0, qa[kk], b[0], b[1]);
+          mma16816(acc1, qa[kk], b[2], b[3]);
+        }
       }
     }
     // mask keys past the split end (last group only)

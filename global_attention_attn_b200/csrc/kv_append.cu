@@ -1,5 +1,7 @@
 // KV append: rotate the first 64 dims of each new key at its position and
-// store key and value into the ring or paged cache.
+// store key and value into the ring or paged cache.  Cache rows hold the key
+// as dims 0..63 rotated in IEEE fp16 and dims 64..191 in bf16 (the input
+// format), and the value in bf16.
 //
 // Cache layout follows the serving pages: window-sized KV for the sliding
 // layers (gaudi-cookbook "MiMo-V2.6-Flash-RL", "Launch": window-sized KV for

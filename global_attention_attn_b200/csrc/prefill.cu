@@ -18,7 +18,9 @@
 // Roles (192 threads): warp 0 issues TMA loads (Q once per M tile, K/V per key
 // tile, 128-byte swizzled), warp 1 allocates TMEM and issues tcgen05.mma
 // (S = Q K^T into TMEM, double-buffered; O += P V with P read from TMEM), warps
-// 2..5 rotate Q in shared memory (partial RoPE fused into the load), run the
+// 2..5 rotate Q in shared memory (partial RoPE fused into the load; the 64
+// rotated dims are written back as fp16 and contracted by an fp16 MMA, the 128
+// other dims by a bf16 MMA into the same accumulator), run the
 // softmax (exp2 domain, running max with rescale only when it grows by more
 // than 2^8, sink folded into the initial max and sum), write P into TMEM over
 // its S columns, and run the epilogue (O * v_scale / l -> bf16, LSE).
@@ -287,8 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+    constexpr uint32_t idesc_qk_rot = idesc_f32acc(128, BN, 0, 0, 0);  // dims 0..63: fp16 x fp16
+    constexpr uint32_t idesc_qk = idesc_f32acc(128, BN, 0, 0, 1);      // dims 64..191: bf16 x bf16
+    constexpr uint32_t idesc_pv = idesc_f32acc(128, 128, 0, 1, 1);
     int mt = 0, jj = 0;
     bool ok = true;
     auto issue_pv = [&](int jp, bool first) -> bool {
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = sdesc_sw128(qbase + c * Ly::kQChunk + kk * 32, 16, 1024);
               const uint64_t bd = sdesc_sw128(kbase + c * Ly::kKChunk + kk * 32, 16, 1024);
-              tc_mma_ss(tmem + b * kColS1, ad, bd, idesc_qk, (c | kk) ? 1u : 0u);
+              tc_mma_ss(tmem + b * kColS1, ad, bd, c == 0 ? idesc_qk_rot : idesc_qk, (c | kk) ? 1u : 0u);
             }
           tc_commit(s_full(b));
           tc_commit(k_empty(ks));
@@ -498,9 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------- key pre-pass
-// contig: 4 lanes per (row, kv head) write rotated dims 0..63 into ws_k.
-// ext: one warp per (ext row, kv head) writes the full rotated key and value,
-//      halo rows from the ring, new rows from k / v.
+// contig: 4 lanes per (row, kv head) write rotated dims 0..63 (fp16) into ws_k.
+// ext: one warp per (ext row, kv head) writes the full rotated key (dims 0..63
+//      fp16, 64..191 bf16) and the value: halo rows copied from the ring (which
+//      stores the same format), new rows rotated from k / v.
 __global__ void __launch_bounds__(256) rope_k_kernel(const RopeKParams p) {
   const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
   if (p.mode == kModeContig) {

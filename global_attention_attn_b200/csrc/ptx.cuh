@@ -118,12 +118,13 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulate.
-// a_mn / b_mn: 1 = operand is MN-major in shared memory, 0 = K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
+// Instruction descriptor, kind::f16 with fp32 accumulate.  ab_fmt: 1 = bf16 A/B,
+// 0 = fp16 A/B (A and B always share one type).  a_mn / b_mn: 1 = operand is
+// MN-major in shared memory, 0 = K-major.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn, int b_mn, uint32_t ab_fmt = 1) {
   return (1u << 4)                       // D format: f32
-         | (1u << 7)                     // A format: bf16
-         | (1u << 10)                    // B format: bf16
+         | (ab_fmt << 7)                 // A format
+         | (ab_fmt << 10)                // B format
          | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 

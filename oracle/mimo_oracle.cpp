@@ -46,6 +46,16 @@ inline double bf16_to_double(uint16_t b) {
   return double(f);
 }
 
+// IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
+inline double f16_to_double(uint16_t h) {
+  const int sign = (h >> 15) & 1, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+  double v;
+  if (e == 0) v = std::ldexp(double(f), -24);                       // zero / subnormal
+  else if (e == 31) v = f ? NAN : INFINITY;
+  else v = std::ldexp(double(f | 0x400), e - 25);                   // (1 + f/1024) * 2^(e-15)
+  return sign ? -v : v;
+}
+
 }  // namespace
 
 extern "C" {
@@ -56,6 +66,8 @@ extern "C" {
 // below new_pos0[s] come from the cache (stored rotated):
 //   cache_kind 1 (paged): page block_table[s * max_pages + pos / page_size], slot pos % page_size
 //   cache_kind 2 (ring):  entry s * page_size + pos % page_size
+// Cache rows use the library's cache format: key dims < rope_dim are IEEE
+// fp16 bit patterns (the rotated part), the other key dims and the values bf16.
 typedef struct {
   int hq, hkv, dqk, dv, rope_dim;
   double rope_base, softmax_scale, v_scale;
@@ -129,7 +141,7 @@ bool fetch_key(const Ctx& C, int s, int p, int g, double* k, double* v) {
     const uint16_t* kp = L->k_cache + (entry * L->hkv + g) * L->dqk;
     const uint16_t* vp = L->v_cache + (entry * L->hkv + g) * L->dv;
     if (k)
-      for (int i = 0; i < L->dqk; ++i) k[i] = bf16_to_double(kp[i]);
+      for (int i = 0; i < L->dqk; ++i) k[i] = i < L->rope_dim ? f16_to_double(kp[i]) : bf16_to_double(kp[i]);
     if (v)
       for (int i = 0; i < L->dv; ++i) v[i] = bf16_to_double(vp[i]);
     return true;

@@ -370,6 +370,30 @@ def test_varlen_equals_separate_calls():
         np.testing.assert_array_equal(l[cu[i]:cu[i + 1]], li)
 
 
+def test_cache_rows_decode_rotated_dims_as_fp16():
+    """Cache rows hold key dims < rope_dim as IEEE fp16 bit patterns (the library's cache
+    format).  A single cached key at position 0 with no sink: lse = scale * q.k exactly."""
+    hq, hkv, dqk, dv, R = 2, 1, 8, 4, 4
+    # fp16 bit patterns: 0x3C00 = 1.0, 0xC000 = -2.0, 0x7BFF = 65504, 0x0001 = 2^-24 (subnormal)
+    f16 = np.array([0x3C00, 0xC000, 0x7BFF, 0x0001], np.uint16)
+    rest = synth.f64_to_bf16_bits(np.array([0.5, -1.5, 3.0, 0.25]))
+    kc = np.zeros((1, 4, hkv, dqk), np.uint16)
+    kc[0, 0, 0, :4] = f16
+    kc[0, 0, 0, 4:] = rest
+    vc = np.zeros((1, 4, hkv, dv), np.uint16)
+    vc[0, 0, 0] = synth.f64_to_bf16_bits(np.array([1.0, 2.0, 3.0, 4.0]))
+    q = synth.f64_to_bf16_bits(np.array([[1.0, 1.0, 1.0, 2.0 ** 10, 1.0, 1.0, 1.0, 1.0],
+                                         [0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 1.0]])).reshape(1, hq, dqk)
+    o, l = oracle.attention(q=q, hq=hq, hkv=hkv, dqk=dqk, dv=dv, rope_dim=R, rope_base=10.0, softmax_scale=0.5,
+                            v_scale=0.707, window=0, sink=None, q_row0=[0], q_len=[1], q_pos0=[0], sel_seq=[0],
+                            sel_row=[0], new_pos0=[1], new_len=[0], cache_kind=2, k_cache=kc, v_cache=vc,
+                            page_size=4)
+    k = [1.0, -2.0, 65504.0, 2.0 ** -24, 0.5, -1.5, 3.0, 0.25]
+    assert l[0, 0] == 0.5 * (1.0 - 2.0 + 65504.0 + 2.0 ** -14 + 0.5 - 1.5 + 3.0 + 0.25)
+    assert l[0, 1] == 0.5 * 0.25
+    np.testing.assert_array_equal(o[0, 0], 0.707 * np.array([1.0, 2.0, 3.0, 4.0]))
+
+
 def test_kv_append_oracle():
     k = bf16(30, (5, 2, 192))
     v = bf16(31, (5, 2, 128))

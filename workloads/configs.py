@@ -6,8 +6,9 @@ heads, 192-dim Q/K, 128-dim V, partial RoPE on 64 dims, sliding-window layers
 with window 128, 8 KV heads, RoPE base 1e4 and a per-head sink; global layers
 with 4 KV heads and RoPE base 1e7.  All tensors are bf16 ~N(0,1) (uint16 bit
 patterns), sinks are fp32 ~N(0,1).  Cached keys are synthetic values that are
-treated as already rotated.  This module draws numbers and lays them out; it
-computes nothing of the attention itself.
+treated as already rotated and are laid out in the library's cache format
+(key dims 0..63 as IEEE fp16, dims 64..191 and values as bf16).  This module
+draws numbers and lays them out; it computes nothing of the attention itself.
 """
 from __future__ import annotations
 
@@ -75,6 +76,28 @@ def _normal_bf16_parallel(key: int, shape) -> np.ndarray:
 
 def bf16_normal(seed: int, tag: int, shape) -> np.ndarray:
     return _normal_bf16_parallel(synth.stream_seed(seed, tag), shape)
+
+
+def cached_keys(seed: int, tag: int, shape) -> np.ndarray:
+    """~N(0,1) key rows [..., 192] in the cache format: dims 0..63 (the rotated part)
+    as IEEE fp16 bit patterns, dims 64..191 as bf16 bit patterns."""
+    assert shape[-1] == DQK
+    rows = int(np.prod(shape[:-1]))
+    out = np.empty((rows, DQK), dtype=np.uint16)
+    step = 1 << 16
+    key = synth.stream_seed(seed, tag)
+
+    def work(lo):
+        hi = min(rows, lo + step)
+        x = synth.normal_f64(synth.stream_seed(key, lo // step), (hi - lo) * DQK).reshape(hi - lo, DQK)
+        out[lo:hi, :ROPE_DIM] = synth.f64_to_f16_bits(x[:, :ROPE_DIM])
+        out[lo:hi, ROPE_DIM:] = synth.f64_to_bf16_bits(x[:, ROPE_DIM:])
+
+    starts = list(range(0, rows, step))
+    nthr = max(1, min(len(starts), len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(nthr) as ex:
+        list(ex.map(work, starts))
+    return out.reshape(shape)
 
 
 @dataclass
@@ -204,12 +227,12 @@ def config3(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536)) -> 
         ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
     Ls = swa_layer(synth.normal_f32(synth.stream_seed(seed, 4), (HQ,)))
     swa = Decode(Ls, bf16_normal(seed, 1, (B, HQ, DQK)), ctx,
-                 bf16_normal(seed, 2, (B, RING, 8, DQK)), bf16_normal(seed, 3, (B, RING, 8, DV)),
+                 cached_keys(seed, 2, (B, RING, 8, DQK)), bf16_normal(seed, 3, (B, RING, 8, DV)),
                  name=f"swa_decode_b{B}_ring128")
     bt, pool = paged_layout(seed, 10, ctx)
     Lg = global_layer()
     glb = Decode(Lg, bf16_normal(seed, 11, (B, HQ, DQK)), ctx,
-                 bf16_normal(seed, 12, (pool, PAGE, 4, DQK)), bf16_normal(seed, 13, (pool, PAGE, 4, DV)),
+                 cached_keys(seed, 12, (pool, PAGE, 4, DQK)), bf16_normal(seed, 13, (pool, PAGE, 4, DV)),
                  block_table=bt, name=f"global_decode_b{B}_paged128")
     return swa, glb
 
@@ -234,7 +257,7 @@ def config4(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int = 8192,
     vc = np.zeros((pool, PAGE, 4, DV), np.uint16)
     # the prefix positions hold synthetic (already rotated) keys; the chunk's slots stay zero
     npre = (prefix + PAGE - 1) // PAGE
-    pk = bf16_normal(seed, 12, (npre * PAGE, 4, DQK))
+    pk = cached_keys(seed, 12, (npre * PAGE, 4, DQK))
     pv = bf16_normal(seed, 13, (npre * PAGE, 4, DV))
     for i in range(npre):
         n = min(PAGE, prefix - i * PAGE)
@@ -248,7 +271,7 @@ def config4(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int = 8192,
     ring_k = np.zeros((1, RING, 8, DQK), np.uint16)
     ring_v = np.zeros((1, RING, 8, DV), np.uint16)
     tail = min(prefix, RING)
-    tk = bf16_normal(seed, 25, (tail, 8, DQK))
+    tk = cached_keys(seed, 25, (tail, 8, DQK))
     tv = bf16_normal(seed, 26, (tail, 8, DV))
     for j in range(tail):
         p = prefix - tail + j

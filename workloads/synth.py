@@ -78,6 +78,11 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return (b >> np.uint32(16)).astype(np.uint16)
 
 
+def f64_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """float64 -> IEEE fp16 (numpy's round-to-nearest-even) as uint16 bit patterns."""
+    return np.ascontiguousarray(x).astype(np.float16).view(np.uint16)
+
+
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
