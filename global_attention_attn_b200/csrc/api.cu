@@ -358,6 +358,7 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
     if ((rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, hkv, kDv, 1, BN))) return rc;
   }
   p.num_seqs = a->num_seqs;
+  p.seq_base = 0;
   p.total_q = a->total_q;
   p.hkv = hkv;
   p.mode = mode;
@@ -399,8 +400,18 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   // upper bound of M tiles: ceil(total_q / R) + num_seqs partial tiles, times KV heads
   const long work = (long(a->total_q) / R + a->num_seqs + 1) * hkv;
   const int grid = int(work < d.sms ? work : d.sms);
-  cudaError_t e = launch_prefill(p, kind, grid, st);
-  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  // one launch per group of at most 256 sequences (the kernel keeps a per-sequence table in shared memory)
+  for (int s0 = 0; s0 < a->num_seqs; s0 += kPrefillMaxSeqsPerLaunch) {
+    PrefillParams q = p;
+    q.seq_base = s0;
+    q.num_seqs = a->num_seqs - s0 < kPrefillMaxSeqsPerLaunch ? a->num_seqs - s0 : kPrefillMaxSeqsPerLaunch;
+    q.cu_q = a->cu_seqlens_q + s0;
+    q.cu_k = a->cu_seqlens_k ? a->cu_seqlens_k + s0 : nullptr;
+    q.cache_lens = a->cache_lens ? a->cache_lens + s0 : nullptr;
+    q.block_table = a->block_table ? a->block_table + long(s0) * a->max_pages : nullptr;
+    cudaError_t e = launch_prefill(q, kind, grid, st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  }
   return MIMO_OK;
 }
 

@@ -53,4 +53,18 @@ __device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int
   }
 }
 
+// Same rotation with precomputed (cos, sin) pairs: cs[i] for frequency 8u+i.
+__device__ __forceinline__ void rope_chunk_pair_cs(uint4& lo, uint4& hi, const float2* cs) {
+  uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float x0 = lo_bf16(a[w]), x1 = hi_bf16(a[w]);
+    const float y0 = lo_bf16(b[w]), y1 = hi_bf16(b[w]);
+    const float2 t0 = cs[2 * w], t1 = cs[2 * w + 1];
+    a[w] = pack2_f16(x0 * t0.x - y0 * t0.y, x1 * t1.x - y1 * t1.y);
+    b[w] = pack2_f16(y0 * t0.x + x0 * t0.y, y1 * t1.x + x1 * t1.y);
+  }
+}
+
 }  // namespace mimo

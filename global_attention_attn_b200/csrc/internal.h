@@ -70,6 +70,7 @@ struct PrefillParams {
   CUtensorMap tm_k12;  // key dims 64..191 source (x = 64, 128), box {64, 1, BN}
   CUtensorMap tm_v;    // value source (x = 0, 64), box {64, 1, BN}
   int num_seqs, total_q, hkv, mode, window;
+  int seq_base;  // index of this launch's first sequence in the whole batch (launches take <= 256)
   const int32_t* cu_q;
   const int32_t* cu_k;
   const int32_t* cache_lens;
@@ -105,6 +106,7 @@ cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s);
 // kind 0: sliding window (G=8 heads x 16 rows, one 144-key tile); kind 1: global (G=16 x 8 rows, 128-key tiles)
 cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s);
 int prefill_rows_per_tile(int kind);
+constexpr int kPrefillMaxSeqsPerLaunch = 256;
 int prefill_key_tile(int kind);
 
 }  // namespace mimo

@@ -54,10 +54,12 @@ struct Cfg<1> {  // global (or any window wider than 129)
   static constexpr int G = 16, R = 8, BN = 128, NQ = 1, NK = 2, NV = 2;
 };
 
+constexpr int kMaxSeqs = kPrefillMaxSeqsPerLaunch;  // sequences per launch (the host splits larger batches)
+
 template <int KIND>
 struct Layout {
   using C = Cfg<KIND>;
-  static constexpr int kQChunk = 128 * 128;          // 128 rows x 64 dims bf16
+  static constexpr int kQChunk = 128 * 128;          // 128 rows x 64 dims, 2-byte elements
   static constexpr int kQStage = 3 * kQChunk;
   static constexpr int kKChunk = C::BN * 128;
   static constexpr int kKStage = 3 * kKChunk;
@@ -67,10 +69,14 @@ struct Layout {
   static constexpr int kOffK = kOffQ + C::NQ * kQStage;
   static constexpr int kOffV = kOffK + C::NK * kKStage;
   static constexpr int kOffBar = kOffV + C::NV * kVStage;
-  static constexpr int kNumBars = 3 * C::NQ + 2 * C::NK + 2 * C::NV + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kNumBars = 3 * C::NQ + 2 * C::NK + 2 * C::NV + 2 + 2 + 1 + 1 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kOffSeq = kOffMisc + 16;                       // int [6][kMaxSeqs + 1]
+  static constexpr int kOffSink = kOffSeq + 6 * (kMaxSeqs + 1) * 4;   // float [64], log2 units
+  static constexpr int kOffCS = kOffSink + 64 * 4;                    // float2 [R][32] cos/sin of a tile
+  static constexpr int kBytes = kOffCS + C::R * 32 * 8;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 struct TileInfo {
@@ -82,61 +88,90 @@ struct TileInfo {
   int krow_base, kpos_base;  // contiguous key sources: row of position kpos_base
 };
 
-// Warp-collective: maps work item w to (sequence, tile, kv head).  Tiles of a
-// sequence are ordered longest-first for global attention.
+// Per-CTA copy of the per-sequence quantities the roles need for every tile.
+struct SeqTable {
+  int* tile_start;  // [B + 1] exclusive prefix of M tiles per sequence
+  int* q0;          // cu_seqlens_q[s]
+  int* qlen;
+  int* clen;        // cache_lens[s]
+  int* k0;          // cu_seqlens_k[s]
+  int* klen;
+};
+
+__device__ __forceinline__ SeqTable seq_table(uint8_t* base) {
+  int* a = reinterpret_cast<int*>(base);
+  constexpr int n = kMaxSeqs + 1;
+  return SeqTable{a, a + n, a + 2 * n, a + 3 * n, a + 4 * n, a + 5 * n};
+}
+
+// One warp fills the table.
 template <int KIND>
-__device__ __forceinline__ bool locate(const PrefillParams& p, int w, TileInfo& T) {
+__device__ __forceinline__ void fill_seq_table(const PrefillParams& p, const SeqTable& S) {
   constexpr int R = Cfg<KIND>::R;
   const int lane = threadIdx.x & 31;
-  const int tt = w / p.hkv;
   int base = 0;
   for (int s0 = 0; s0 < p.num_seqs; s0 += 32) {
     const int s = s0 + lane;
     int n = 0;
-    if (s < p.num_seqs) n = (p.cu_q[s + 1] - p.cu_q[s] + R - 1) / R;
+    if (s < p.num_seqs) {
+      const int q0 = p.cu_q[s], ql = p.cu_q[s + 1] - q0;
+      n = (ql + R - 1) / R;
+      S.q0[s] = q0;
+      S.qlen[s] = ql;
+      S.clen[s] = p.cache_lens ? p.cache_lens[s] : 0;
+      S.k0[s] = p.cu_k ? p.cu_k[s] : 0;
+      S.klen[s] = p.cu_k ? p.cu_k[s + 1] - p.cu_k[s] : 0;
+    }
     int incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    if (tt < base + total) {
-      const unsigned hit = __ballot_sync(0xffffffffu, tt < base + incl && tt >= base + incl - n);
-      const int src = __ffs(hit) - 1;
-      T.s = s0 + src;
-      T.ntiles = __shfl_sync(0xffffffffu, n, src);
-      const int excl = __shfl_sync(0xffffffffu, incl - n, src);
-      int t = tt - base - excl;
-      if (KIND == 1) t = T.ntiles - 1 - t;
-      T.t = t;
-      T.g = w % p.hkv;
-      const int q0 = p.cu_q[T.s], qlen = p.cu_q[T.s + 1] - q0;
-      const int clen = p.cache_lens ? p.cache_lens[T.s] : 0;
-      const int klen = p.cu_k ? p.cu_k[T.s + 1] - p.cu_k[T.s] : 0;
-      const int ctx = clen + klen;
-      T.q_row0 = q0 + t * R;
-      T.rows_valid = min(R, qlen - t * R);
-      T.qpos0 = ctx - qlen + t * R;
-      if (p.mode == kModeContig) {
-        T.key_lo = clen;
-        T.krow_base = p.cu_k[T.s];
-        T.kpos_base = clen;
-      } else if (p.mode == kModeExt) {
-        T.key_lo = max(0, clen - 128);
-        T.krow_base = p.cu_k[T.s] + 128 * T.s;
-        T.kpos_base = clen - 128;
-      } else {
-        T.key_lo = 0;
-        T.krow_base = 0;
-        T.kpos_base = 0;
-      }
-      if (ctx < qlen && lane == 0 && t == 0 && T.g == 0) atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
-      return true;
-    }
-    base += total;
+    if (s < p.num_seqs) S.tile_start[s] = base + incl - n;
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  return false;
+  if (lane == 0) S.tile_start[p.num_seqs] = base;
+}
+
+// Maps work item w to (sequence, tile, kv head) from the shared table; any
+// thread may call it.  Tiles of a sequence are ordered longest-first for
+// global attention.
+template <int KIND>
+__device__ __forceinline__ bool locate(const PrefillParams& p, const SeqTable& S, int w, TileInfo& T) {
+  constexpr int R = Cfg<KIND>::R;
+  const int tt = w / p.hkv;
+  if (tt >= S.tile_start[p.num_seqs]) return false;
+  int lo = 0, hi = p.num_seqs;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (S.tile_start[mid] <= tt) lo = mid; else hi = mid;
+  }
+  T.s = lo;
+  T.ntiles = S.tile_start[lo + 1] - S.tile_start[lo];
+  int t = tt - S.tile_start[lo];
+  if (KIND == 1) t = T.ntiles - 1 - t;
+  T.t = t;
+  T.g = w % p.hkv;
+  const int qlen = S.qlen[lo], clen = S.clen[lo];
+  const int ctx = clen + S.klen[lo];
+  T.q_row0 = S.q0[lo] + t * R;
+  T.rows_valid = min(R, qlen - t * R);
+  T.qpos0 = ctx - qlen + t * R;
+  if (p.mode == kModeContig) {
+    T.key_lo = clen;
+    T.krow_base = S.k0[lo];
+    T.kpos_base = clen;
+  } else if (p.mode == kModeExt) {
+    T.key_lo = max(0, clen - 128);
+    T.krow_base = S.k0[lo] + 128 * (p.seq_base + lo);
+    T.kpos_base = clen - 128;
+  } else {
+    T.key_lo = 0;
+    T.krow_base = 0;
+    T.kpos_base = 0;
+  }
+  return true;
 }
 
 // Key tiles of an M tile: [j_lo, j_lo + n) with tile j starting at position key_tile_start(j).
@@ -183,8 +218,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const uint32_t pv_done = bar0 + 8 * (3 * NQ + 2 * NK + 2 * NV + 4);
   const uint32_t o_empty = pv_done + 8;
   const uint32_t drain = pv_done + 16;
+  const uint32_t cs_ready = pv_done + 24;  // the softmax warps' cos/sin table is written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::kOffMisc + 4);
+  const SeqTable S = seq_table(smem + Ly::kOffSeq);
+  float* sink_l2 = reinterpret_cast<float*>(smem + Ly::kOffSink);
+  float2* cs = reinterpret_cast<float2*>(smem + Ly::kOffCS);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NQ; ++i) {
@@ -207,13 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     mbar_init(pv_done, 1);
     mbar_init(o_empty, 128);
     mbar_init(drain, 1);
+    mbar_init(cs_ready, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 0) fill_seq_table<KIND>(p, S);
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  if (threadIdx.x >= 64 && threadIdx.x < 128)
+    sink_l2[threadIdx.x - 64] = p.sink ? p.sink[threadIdx.x - 64] * kLog2e : -INFINITY;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -221,88 +264,96 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   unsigned* status = p.status;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch(&p.tm_q);
-      tma_prefetch(&p.tm_k0);
-      tma_prefetch(&p.tm_k12);
-      tma_prefetch(&p.tm_v);
-    }
-    int mt = 0, jj = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; ok; w += gridDim.x) {
-      TileInfo T;
-      if (!locate<KIND>(p, w, T)) break;
-      const int qs = mt % NQ;
-      if (mt >= NQ) ok = mbar_wait(q_empty(qs), ((mt / NQ) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
-      if (!ok) break;
+    // ------------------------------------------------------------ TMA producers
+    // lane 0 streams Q tiles, lane 1 K tiles, lane 2 V tiles, each at its own pace.
+    if (lane < 3) {
       if (lane == 0) {
-        const uint32_t qdst = sbase + Ly::kOffQ + qs * Ly::kQStage;
-        mbar_expect_tx(q_full(qs), Ly::kQStage);
-        for (int c = 0; c < 3; ++c) tma_load_3d(qdst + c * Ly::kQChunk, &p.tm_q, q_full(qs), 64 * c, T.g * G, T.q_row0);
+        tma_prefetch(&p.tm_q);
+        tma_prefetch(&p.tm_k0);
+        tma_prefetch(&p.tm_k12);
+        tma_prefetch(&p.tm_v);
       }
-      int j_lo, nkv;
-      key_tiles<KIND>(p, T, &j_lo, &nkv);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int kt0 = key_tile_start<KIND>(T, j_lo + j);
-        int row;
-        if (p.mode == kModePaged) {
-          const int pi = j_lo + j;
-          int page = pi < p.max_pages ? p.block_table[long(T.s) * p.max_pages + pi] : -1;
-          if (page < 0 || page >= p.num_pages) {
-            if (lane == 0) atomicOr(status, MIMO_STATUS_BAD_INDEX);
-            page = 0;
-          }
-          row = page * 128;
+      int mt = 0, jj = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok; w += gridDim.x) {
+        TileInfo T;
+        if (!locate<KIND>(p, S, w, T)) break;
+        if (lane == 0) {
+          const int qs = mt % NQ;
+          if (mt >= NQ) ok = mbar_wait(q_empty(qs), ((mt / NQ) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+          if (!ok) break;
+          const uint32_t qdst = sbase + Ly::kOffQ + qs * Ly::kQStage;
+          mbar_expect_tx(q_full(qs), Ly::kQStage);
+          for (int c = 0; c < 3; ++c)
+            tma_load_3d(qdst + c * Ly::kQChunk, &p.tm_q, q_full(qs), 64 * c, T.g * G, T.q_row0);
         } else {
-          row = T.krow_base + (kt0 - T.kpos_base);
+          int j_lo, nkv;
+          key_tiles<KIND>(p, T, &j_lo, &nkv);
+          for (int j = 0; j < nkv && ok; ++j, ++jj) {
+            const int kt0 = key_tile_start<KIND>(T, j_lo + j);
+            int row;
+            if (p.mode == kModePaged) {
+              const int pi = j_lo + j;
+              int page = pi < p.max_pages ? p.block_table[long(T.s) * p.max_pages + pi] : -1;
+              if (page < 0 || page >= p.num_pages) {
+                if (lane == 1) atomicOr(status, MIMO_STATUS_BAD_INDEX);
+                page = 0;
+              }
+              row = page * 128;
+            } else {
+              row = T.krow_base + (kt0 - T.kpos_base);
+            }
+            if (lane == 1) {
+              const int ks = jj % NK;
+              if (jj >= NK) ok = mbar_wait(k_empty(ks), ((jj / NK) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+              if (!ok) break;
+              const uint32_t kdst = sbase + Ly::kOffK + ks * Ly::kKStage;
+              mbar_expect_tx(k_full(ks), Ly::kKStage);
+              tma_load_3d(kdst, &p.tm_k0, k_full(ks), 0, T.g, row);
+              tma_load_3d(kdst + Ly::kKChunk, &p.tm_k12, k_full(ks), 64, T.g, row);
+              tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full(ks), 128, T.g, row);
+            } else {
+              const int vs = jj % NV;
+              if (jj >= NV) ok = mbar_wait(v_empty(vs), ((jj / NV) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+              if (!ok) break;
+              const uint32_t vdst = sbase + Ly::kOffV + vs * Ly::kVStage;
+              mbar_expect_tx(v_full(vs), Ly::kVStage);
+              tma_load_3d(vdst, &p.tm_v, v_full(vs), 0, T.g, row);
+              tma_load_3d(vdst + Ly::kVChunk, &p.tm_v, v_full(vs), 64, T.g, row);
+            }
+          }
         }
-        const int ks = jj % NK;
-        if (jj >= NK) ok = mbar_wait(k_empty(ks), ((jj / NK) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t kdst = sbase + Ly::kOffK + ks * Ly::kKStage;
-          mbar_expect_tx(k_full(ks), Ly::kKStage);
-          tma_load_3d(kdst, &p.tm_k0, k_full(ks), 0, T.g, row);
-          tma_load_3d(kdst + Ly::kKChunk, &p.tm_k12, k_full(ks), 64, T.g, row);
-          tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full(ks), 128, T.g, row);
-        }
-        const int vs = jj % NV;
-        if (jj >= NV) ok = mbar_wait(v_empty(vs), ((jj / NV) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t vdst = sbase + Ly::kOffV + vs * Ly::kVStage;
-          mbar_expect_tx(v_full(vs), Ly::kVStage);
-          tma_load_3d(vdst, &p.tm_v, v_full(vs), 0, T.g, row);
-          tma_load_3d(vdst + Ly::kVChunk, &p.tm_v, v_full(vs), 64, T.g, row);
-        }
-        ++jj;
+        ++mt;
       }
-      ++mt;
+      if (!ok) {
+        // let copies already in flight land before the CTA leaves
+        int dummy = 0;
+        for (int i = 0; i < NQ; ++i) mbar_wait(q_full(i), 0, &dummy, nullptr, 0, 50000000ull);
+        for (int i = 0; i < NK; ++i) mbar_wait(k_full(i), 0, &dummy, nullptr, 0, 50000000ull);
+        for (int i = 0; i < NV; ++i) mbar_wait(v_full(i), 0, &dummy, nullptr, 0, 50000000ull);
+      }
     }
-    if (!ok && lane == 0) {
-      // let copies already in flight land before the CTA leaves
-      int dummy = 0;
-      for (int i = 0; i < NQ; ++i) mbar_wait(q_full(i), 0, &dummy, nullptr, 0, 50000000ull);
-      for (int i = 0; i < NK; ++i) mbar_wait(k_full(i), 0, &dummy, nullptr, 0, 50000000ull);
-      for (int i = 0; i < NV; ++i) mbar_wait(v_full(i), 0, &dummy, nullptr, 0, 50000000ull);
-    }
+    __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_qk_rot = idesc_f32acc(128, BN, 0, 0, 0);  // dims 0..63: fp16 x fp16
-    constexpr uint32_t idesc_qk = idesc_f32acc(128, BN, 0, 0, 1);      // dims 64..191: bf16 x bf16
-    constexpr uint32_t idesc_pv = idesc_f32acc(128, 128, 0, 1, 1);
-    int mt = 0, jj = 0;
-    bool ok = true;
-    auto issue_pv = [&](int jp, bool first) -> bool {
-      const int b = jp & 1;
-      if (!mbar_wait(p_full(b), (jp >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
-      const int vs = jp % NV;
-      if (!mbar_wait(v_full(vs), (jp / NV) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
-      if (first && mt > 0 && !mbar_wait(o_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))
-        return false;
-      tc_fence_after();
-      if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (lane 0)
+    // Issue order over the continuous stream of key tiles: QK(jj), then PV(jj-1),
+    // so the next M tile's QK^T runs while the current tile's softmax finishes.
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk_rot = idesc_f32acc(128, BN, 0, 0, 0);  // dims 0..63: fp16 x fp16
+      constexpr uint32_t idesc_qk = idesc_f32acc(128, BN, 0, 0, 1);      // dims 64..191: bf16 x bf16
+      constexpr uint32_t idesc_pv = idesc_f32acc(128, 128, 0, 1, 1);
+      int mt = 0, jj = 0;
+      bool ok = true;
+      int pend_jj = -1, pend_mt = 0;
+      bool pend_first = false;
+      auto issue_pv = [&](int jp, bool first, int mtp) -> bool {
+        const int b = jp & 1;
+        if (!mbar_wait(p_full(b), (jp >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        const int vs = jp % NV;
+        if (!mbar_wait(v_full(vs), (jp / NV) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        if (first && mtp > 0 && !mbar_wait(o_empty, (mtp - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))
+          return false;
+        tc_fence_after();
         const uint32_t vbase = sbase + Ly::kOffV + vs * Ly::kVStage;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -311,25 +362,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         }
         tc_commit(v_empty(vs));
         tc_commit(pv_done);
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int w = blockIdx.x; ok; w += gridDim.x) {
-      TileInfo T;
-      if (!locate<KIND>(p, w, T)) break;
-      const int qs = mt % NQ;
-      if (!(ok = mbar_wait(q_rot(qs), (mt / NQ) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
-      tc_fence_after();
-      int j_lo, nkv;
-      key_tiles<KIND>(p, T, &j_lo, &nkv);
-      const uint32_t qbase = sbase + Ly::kOffQ + qs * Ly::kQStage;
-      for (int j = 0; j < nkv; ++j) {
-        const int ks = jj % NK;
-        if (!(ok = mbar_wait(k_full(ks), (jj / NK) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+        return true;
+      };
+      for (int w = blockIdx.x; ok; w += gridDim.x) {
+        TileInfo T;
+        if (!locate<KIND>(p, S, w, T)) break;
+        const int qs = mt % NQ;
+        if (!(ok = mbar_wait(q_rot(qs), (mt / NQ) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
         tc_fence_after();
-        const int b = jj & 1;
-        if (lane == 0) {
+        int j_lo, nkv;
+        key_tiles<KIND>(p, T, &j_lo, &nkv);
+        const uint32_t qbase = sbase + Ly::kOffQ + qs * Ly::kQStage;
+        for (int j = 0; j < nkv; ++j) {
+          const int ks = jj % NK;
+          if (!(ok = mbar_wait(k_full(ks), (jj / NK) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          tc_fence_after();
+          const int b = jj & 1;
           const uint32_t kbase = sbase + Ly::kOffK + ks * Ly::kKStage;
 #pragma unroll
           for (int c = 0; c < 3; ++c)
@@ -342,55 +390,84 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           tc_commit(s_full(b));
           tc_commit(k_empty(ks));
           if (j == nkv - 1) tc_commit(q_empty(qs));
+          if (pend_jj >= 0 && !(ok = issue_pv(pend_jj, pend_first, pend_mt))) break;
+          pend_jj = jj;
+          pend_first = (j == 0);
+          pend_mt = mt;
+          ++jj;
         }
-        __syncwarp();
-        if (j > 0 && !(ok = issue_pv(jj - 1, j == 1))) break;
-        ++jj;
+        if (!ok) break;
+        ++mt;
       }
-      if (!ok) break;
-      if (!(ok = issue_pv(jj - 1, nkv == 1))) break;
-      ++mt;
+      if (ok && pend_jj >= 0) ok = issue_pv(pend_jj, pend_first, pend_mt);
+      if (!ok) {
+        int dummy = 0;
+        tc_commit(drain);
+        mbar_wait(drain, 0, &dummy, nullptr, 0, 50000000ull);
+      }
     }
-    if (!ok && lane == 0) {
-      int dummy = 0;
-      tc_commit(drain);
-      mbar_wait(drain, 0, &dummy, nullptr, 0, 50000000ull);
-    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ RoPE + softmax + epilogue
+    const int tid = threadIdx.x - 64;  // 0..127
     const int quad = warp & 3;
     const int m = quad * 32 + lane;  // TMEM lane = M row
     const int r = m / G, hq = m % G;
     const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16);
     const float c_log2 = p.scale_log2;
+
+    // The four softmax warps take every decision together: a wait that fails in one
+    // lane fails for the whole warp, so warp-collective tcgen05 ops never diverge.
+    auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
+    };
+    int n_rot = 0;
+    // Partial RoPE of M tile T in Q stage qs: the R x 32 cos/sin pairs are computed
+    // once per tile (the G heads of a position share them), then each thread
+    // rotates dims 0..63 of its row in place (128-byte swizzled rows) to fp16.
+    // The table is free to overwrite here: every thread read the previous one
+    // before arriving on q_rot, and this thread passed an s_full since.
+    auto rotate_q = [&](const TileInfo& T, int qs) -> bool {
+#pragma unroll
+      for (int e = tid; e < R * 32; e += 128) {
+        const int rr = e >> 5, j = e & 31;
+        const int pos = rr < T.rows_valid ? T.qpos0 + rr : 0;
+        float c, s;
+        rope_cos_sin(pos, p.rope.inv_freq[j], &c, &s);
+        cs[e] = make_float2(c, s);
+      }
+      mbar_arrive(cs_ready);
+      if (!wait_w(cs_ready, n_rot & 1)) return false;
+      ++n_rot;
+      uint8_t* row = smem + Ly::kOffQ + qs * Ly::kQStage + m * 128;
+      const int sw = m & 7;
+      const float2* csr = cs + r * 32;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint4* plo = reinterpret_cast<uint4*>(row + ((u ^ sw) << 4));
+        uint4* phi = reinterpret_cast<uint4*>(row + (((u + 4) ^ sw) << 4));
+        uint4 lo = *plo, hi = *phi;
+        rope_chunk_pair_cs(lo, hi, csr + 8 * u);
+        *plo = lo;
+        *phi = hi;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_rot(qs));
+      return true;
+    };
+
     int mt = 0, jj = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok; w += gridDim.x) {
-      TileInfo T;
-      if (!locate<KIND>(p, w, T)) break;
-      const int qs = mt % NQ;
-      if (!(ok = mbar_wait(q_full(qs), (mt / NQ) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+    int w = blockIdx.x;
+    TileInfo T;
+    bool have = locate<KIND>(p, S, w, T);
+    if (have) ok = wait_w(q_full(0), 0) && rotate_q(T, 0);
+    while (have && ok) {
       const bool row_valid = r < T.rows_valid;
       const int qp = T.qpos0 + r;
-      {  // partial RoPE on dims 0..63 of this row (chunk 0, 128-byte swizzled rows)
-        uint8_t* row = smem + Ly::kOffQ + qs * Ly::kQStage + m * 128;
-        const int sw = m & 7;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4* plo = reinterpret_cast<uint4*>(row + ((u ^ sw) << 4));
-          uint4* phi = reinterpret_cast<uint4*>(row + (((u + 4) ^ sw) << 4));
-          uint4 lo = *plo, hi = *phi;
-          rope_chunk_pair(lo, hi, u, row_valid ? qp : 0, p.rope);
-          *plo = lo;
-          *phi = hi;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(q_rot(qs));
-      }
       const int head = T.g * G + hq;
-      const bool has_sink = p.sink != nullptr;
-      float m_run = has_sink ? p.sink[head] * kLog2e : -INFINITY;
-      float l_run = has_sink ? 1.f : 0.f;
+      float m_run = sink_l2[head];
+      float l_run = p.sink ? 1.f : 0.f;
       // visible key positions of this row: [vis_lo, vis_hi]
       const int vis_hi = row_valid ? qp : -0x40000000;
       const int vis_lo = max(T.key_lo, p.window > 0 ? qp - p.window + 1 : -0x40000000);
@@ -399,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int qlast = T.qpos0 + T.rows_valid - 1;
       for (int j = 0; j < nkv; ++j) {
         const int b = jj & 1;
-        if (!(ok = mbar_wait(s_full(b), (jj >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+        if (!(ok = wait_w(s_full(b), (jj >> 1) & 1))) break;
         tc_fence_after();
         uint32_t sr[BN];
 #pragma unroll
@@ -423,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           }
         }
         const float mt_l2 = mx * c_log2;
-        if (j > 0 && !(ok = mbar_wait(pv_done, (jj - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+        if (j > 0 && !(ok = wait_w(pv_done, (jj - 1) & 1))) break;
         const float m_new = fmaxf(m_run, mt_l2);
         float alpha = 1.f;
         const bool resc = m_new > m_run + 8.f;
@@ -464,8 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         ++jj;
       }
       if (!ok) break;
+      // ---- rotate the next tile's Q before this tile's epilogue, so its QK^T overlaps
+      w += gridDim.x;
+      TileInfo Tn;
+      const bool have_next = locate<KIND>(p, S, w, Tn);
+      if (have_next) {
+        const int qs = (mt + 1) % NQ;
+        if (!(ok = wait_w(q_full(qs), ((mt + 1) / NQ) & 1) && rotate_q(Tn, qs))) break;
+      }
       // ---- epilogue
-      if (!(ok = mbar_wait(pv_done, (jj - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+      if (!(ok = wait_w(pv_done, (jj - 1) & 1))) break;
       tc_fence_after();
       const float sc = p.v_scale / l_run;
       uint16_t* orow = p.out + (long(T.q_row0 + r) * kHq + head) * kDv;
@@ -489,6 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(o_empty);
       ++mt;
+      T = Tn;
+      have = have_next;
     }
   }
 

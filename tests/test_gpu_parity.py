@@ -150,6 +150,13 @@ def test_prefill_swa_edges(lens):
     check_prefill(make_prefill(lens, 8, 1e4, 128, True, 200 + sum(lens)), what=f"swa {lens}")
 
 
+def test_prefill_many_sequences():
+    """More than 256 sequences: the batch is split over several launches."""
+    lens = list((np.arange(300) * 7919) % 37 + 1)
+    check_prefill(make_prefill(lens, 8, 1e4, 128, True, 310), what="swa 300 sequences")
+    check_prefill(make_prefill(lens, 4, 1e7, 0, False, 311), what="global 300 sequences")
+
+
 def test_prefill_swa_no_sink():
     check_prefill(make_prefill([513, 77], 8, 1e4, 128, False, 301), what="swa no sink")
 
