@@ -38,7 +38,9 @@ FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) p
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel, from the ncu
 # capture summarised in profiles/ (None until a capture of the current kernel exists).
-TRAFFIC_BYTES = {"prefill_kernel<0>/swa_varlen_prefill": None}
+# Kernel at commit 7c1eebe: 247.6 MB read + 97.9 MB written for 2 x 4096 tokens
+# (profiles/prefill_swa_2x4096_full.md), scaled by tokens to the 40696-token workload.
+TRAFFIC_BYTES = {"prefill_kernel<0>/swa_varlen_prefill": int((247.605504e6 + 97.874432e6) * 40696 / 8192)}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
