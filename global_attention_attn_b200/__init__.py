@@ -34,8 +34,9 @@ SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
 V_SCALE = 0.707
 
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_prefill_workspace_size", "mimo_attn_decode",
-           "mimo_attn_decode_workspace_size", "mimo_kv_append", "mimo_last_error", "mimo_status_poll",
-           "mimo_version")
+           "mimo_attn_decode_workspace_size", "mimo_attn_decode_noalloc", "mimo_kv_append", "mimo_last_error",
+           "mimo_status_poll", "mimo_version")
+DECODE_NOALLOC_MAX_BYTES = 16 << 20
 
 _P = C.c_void_p
 _PI = C.POINTER(C.c_int32)
@@ -95,6 +96,8 @@ def lib():
         L.mimo_attn_decode.restype = C.c_int
         L.mimo_attn_decode_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
         L.mimo_attn_decode_workspace_size.restype = C.c_size_t
+        L.mimo_attn_decode_noalloc.argtypes = [C.POINTER(MimoDecodeArgs), _P]
+        L.mimo_attn_decode_noalloc.restype = C.c_int
         L.mimo_kv_append.argtypes = [C.POINTER(MimoAppendArgs), _P]
         L.mimo_kv_append.restype = C.c_int
         L.mimo_last_error.argtypes = []
@@ -201,6 +204,25 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mimo_attn_decode(C.byref(a), _stream(stream)))
+    return out, lse
+
+
+def mimo_attn_decode_noalloc(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_base: float, window: int,
+                             cache_kind: int, k_cache, v_cache, out, lse=None, block_table=None, num_pages: int = 0,
+                             sink=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None):
+    """Decode that allocates nothing (see mimo_attn_decode_noalloc in include/mimoattn.h): the
+    caller passes the output buffers; the split-KV partials go to the library's static
+    device scratch (16 MiB), so concurrent calls must not overlap on the GPU."""
+    a = MimoDecodeArgs()
+    a.layer = make_layer(num_kv_heads, rope_base, window, sink, softmax_scale, v_scale)
+    a.batch, a.max_seq_len = q.shape[0], int(max_seq_len)
+    a.q, a.seq_lens = _ptr(q), _ptr(seq_lens)
+    a.cache_kind = cache_kind
+    a.k_cache, a.v_cache, a.block_table = _ptr(k_cache), _ptr(v_cache), _ptr(block_table)
+    a.max_pages = 0 if block_table is None else block_table.shape[1]
+    a.num_pages = num_pages
+    a.out, a.lse = _ptr(out), _ptr(lse)
+    _check(lib().mimo_attn_decode_noalloc(C.byref(a), _stream(stream)))
     return out, lse
 
 

@@ -415,6 +415,64 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   return MIMO_OK;
 }
 
+}  // extern "C"
+
+namespace mimo {
+namespace {
+
+// Split-KV partials of mimo_attn_decode_noalloc.  Device code never names it:
+// host code passes the per-device address obtained below.
+static __device__ __align__(256) unsigned char g_decode_scratch[MIMO_DECODE_NOALLOC_MAX_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64];
+
+// Address of this device's copy of g_decode_scratch (looked up once per device,
+// with that device current).  In host code the array's name is only a stand-in.
+int scratch_address(const char* fn, void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(MIMO_ERR_CUDA, "%s: device index %d out of range", fn, dev);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress of the scratch array: %s", fn, cudaGetErrorString(e));
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return MIMO_OK;
+}
+
+}  // namespace
+}  // namespace mimo
+
+extern "C" {
+
+int mimo_attn_decode_noalloc(const mimo_decode_args* a, void* stream) {
+  const char* fn = "mimo_attn_decode_noalloc";
+  if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  if (a->batch > 0 && a->max_seq_len > 0) {
+    const size_t need =
+        mimo_attn_decode_workspace_size(a->batch, a->max_seq_len, a->layer.num_kv_heads, a->layer.window);
+    if (need > MIMO_DECODE_NOALLOC_MAX_BYTES)
+      return fail(MIMO_ERR_WORKSPACE,
+                  "%s: batch %d x max_seq_len %d needs %zu bytes of split-KV partials; the library's static "
+                  "scratch holds %u (use mimo_attn_decode with a caller workspace)",
+                  fn, a->batch, a->max_seq_len, need, unsigned(MIMO_DECODE_NOALLOC_MAX_BYTES));
+  }
+  mimo_decode_args b = *a;
+  b.workspace = nullptr;
+  b.workspace_bytes = 0;
+  if (a->batch > 0) {
+    if (int rc = scratch_address(fn, &b.workspace)) return rc;
+    b.workspace_bytes = MIMO_DECODE_NOALLOC_MAX_BYTES;
+  }
+  return mimo_attn_decode(&b, stream);
+}
+
 int mimo_status_poll(uint32_t* status) {
   const char* fn = "mimo_status_poll";
   if (!status) return fail(MIMO_ERR_INVALID_ARG, "%s: status is NULL", fn);

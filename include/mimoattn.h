@@ -166,6 +166,32 @@ MIMO_API size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int 
 MIMO_API int mimo_attn_decode(const mimo_decode_args* args, void* stream);
 
 /*
+ * Decode for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart: this is a deployment convenience.  Some callers
+ * cannot call cudaMalloc at all: code running inside a CUDA graph capture
+ * region, or runtimes whose only device memory is a fixed arena handed out by
+ * someone else.  For them this entry point behaves exactly like
+ * mimo_attn_decode, except that `workspace` / `workspace_bytes` in the
+ * arguments are ignored: the split-KV partials go to a library-owned device
+ * array of MIMO_DECODE_NOALLOC_MAX_BYTES (16 MiB) that every GPU which loads the
+ * library holds until the process exits.
+ *   - Nothing is allocated: no cudaMalloc / cudaFree, no allocating library call.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current): make that first call
+ *     before any stream capture.
+ *   - Problems whose partials need more than MIMO_DECODE_NOALLOC_MAX_BYTES
+ *     (mimo_attn_decode_workspace_size of the same sizes) are rejected with
+ *     MIMO_ERR_WORKSPACE before anything is enqueued.
+ *   - All calls share the one array, so calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads) race and corrupt each
+ *     other's results; serialise them.  No part of the array needs to start at
+ *     zero: each call writes every partial it later reads.
+ */
+#define MIMO_DECODE_NOALLOC_MAX_BYTES (16u << 20)
+MIMO_API int mimo_attn_decode_noalloc(const mimo_decode_args* args, void* stream);
+
+/*
  * KV append: rotates the first 64 dims of each new key at its position (the
  * layer's RoPE base, angles from float64) and stores key and value (value
  * unscaled) in the cache: ring slot pos % 128 of sequence seq_idx[t], or page
