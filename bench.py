@@ -210,7 +210,7 @@ class Prefill:
         T = self.q.shape[0]
         self.out = torch.empty((T, 64, 128), dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty((T, 64), dtype=torch.float32, device="cuda")
-        n = M.prefill_workspace_size(cfg.num_seqs, self.k.shape[0], L.num_kv_heads, M.MIMO_CACHE_NONE)
+        n = M.prefill_workspace_size(cfg.num_seqs, T, self.k.shape[0], L.num_kv_heads, M.MIMO_CACHE_NONE)
         self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
 
     def __call__(self):
@@ -268,7 +268,7 @@ class Chunked:
             self.ws = None
         else:
             self.start = dev_i32(cfg.start)
-            w = M.prefill_workspace_size(1, n, L.num_kv_heads, M.MIMO_CACHE_RING)
+            w = M.prefill_workspace_size(1, n, n, L.num_kv_heads, M.MIMO_CACHE_RING)
             self.ws = torch.empty(w, dtype=torch.uint8, device="cuda")
 
     def __call__(self):

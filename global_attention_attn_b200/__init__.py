@@ -90,7 +90,7 @@ def lib():
         L = C.CDLL(LIB_PATH)
         L.mimo_attn_prefill.argtypes = [C.POINTER(MimoPrefillArgs), _P]
         L.mimo_attn_prefill.restype = C.c_int
-        L.mimo_attn_prefill_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
+        L.mimo_attn_prefill_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]
         L.mimo_attn_prefill_workspace_size.restype = C.c_size_t
         L.mimo_attn_decode.argtypes = [C.POINTER(MimoDecodeArgs), _P]
         L.mimo_attn_decode.restype = C.c_int
@@ -136,8 +136,8 @@ def make_layer(num_kv_heads: int, rope_base: float, window: int, sink=None, soft
     return L
 
 
-def prefill_workspace_size(num_seqs: int, total_k: int, num_kv_heads: int, cache_kind: int) -> int:
-    return int(lib().mimo_attn_prefill_workspace_size(num_seqs, total_k, num_kv_heads, cache_kind))
+def prefill_workspace_size(num_seqs: int, total_q: int, total_k: int, num_kv_heads: int, cache_kind: int) -> int:
+    return int(lib().mimo_attn_prefill_workspace_size(num_seqs, total_q, total_k, num_kv_heads, cache_kind))
 
 
 def decode_workspace_size(batch: int, max_seq_len: int, num_kv_heads: int, window: int) -> int:
@@ -159,7 +159,7 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
         out = torch.empty((total_q, NUM_Q_HEADS, HEAD_DIM_V), dtype=torch.bfloat16, device=q.device)
     if lse is None and with_lse:
         lse = torch.empty((total_q, NUM_Q_HEADS), dtype=torch.float32, device=q.device)
-    need = prefill_workspace_size(num_seqs, total_k, num_kv_heads, cache_kind)
+    need = prefill_workspace_size(num_seqs, total_q, total_k, num_kv_heads, cache_kind)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     a = MimoPrefillArgs()

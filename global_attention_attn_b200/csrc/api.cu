@@ -139,14 +139,15 @@ const char* mimo_last_error(void) { return g_err; }
 
 const char* mimo_version(void) { return "libmimoattn 0.1 (sm_100a)"; }
 
-size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_k, int num_kv_heads, int cache_kind) {
-  if (num_seqs < 0 || total_k < 0 || num_kv_heads <= 0) return 0;
+size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_q, int total_k, int num_kv_heads, int cache_kind) {
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || num_kv_heads <= 0) return 0;
   if (cache_kind == MIMO_CACHE_PAGED) return 0;
+  const size_t cs = round256(size_t(total_q) * kHalf * 8);  // (cos, sin) per query row and frequency
   if (cache_kind == MIMO_CACHE_RING) {
     const size_t rows = size_t(total_k) + 128 * size_t(num_seqs);
-    return round256(rows * num_kv_heads * kDqk * 2) + round256(rows * num_kv_heads * kDv * 2);
+    return round256(rows * num_kv_heads * kDqk * 2) + round256(rows * num_kv_heads * kDv * 2) + cs;
   }
-  return round256(size_t(total_k) * num_kv_heads * kRope * 2);
+  return round256(size_t(total_k) * num_kv_heads * kRope * 2) + cs;
 }
 
 size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int num_kv_heads, int window) {
@@ -318,7 +319,7 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
       mode = kModeContig;
     }
   }
-  const size_t need = mimo_attn_prefill_workspace_size(a->num_seqs, a->total_k, hkv, a->cache_kind);
+  const size_t need = mimo_attn_prefill_workspace_size(a->num_seqs, a->total_q, a->total_k, hkv, a->cache_kind);
   if (need > 0) {
     if (!a->workspace || a->workspace_bytes < need)
       return fail(MIMO_ERR_WORKSPACE, "%s: workspace of %zu bytes required (got %zu)", fn, need,
@@ -341,6 +342,22 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   if (rc) return rc;
   uint16_t* ws_k = static_cast<uint16_t*>(a->workspace);
   uint16_t* ws_v = nullptr;
+  float2* cs_q = nullptr;
+  if (mode != kModePaged) {
+    const size_t cs_bytes = round256(size_t(a->total_q) * kHalf * 8);
+    cs_q = reinterpret_cast<float2*>(static_cast<char*>(a->workspace) + need - cs_bytes);
+  }
+  if (kind == 0) {
+    // 2-D fp32 table [total_q, 64] (cos, sin interleaved per frequency), box {64, 16}, no swizzle
+    cuuint64_t gdim[2] = {64, cuuint64_t(a->total_q)};
+    cuuint64_t gstride[1] = {64 * 4};
+    cuuint32_t box[2] = {64, cuuint32_t(R)};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(&p.tm_cs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, cs_q, gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MIMO_ERR_CUDA, "%s: cuTensorMapEncodeTiled (cos/sin table) failed (%d)", fn, int(r));
+  }
   if (mode == kModeContig) {
     if ((rc = make_map(fn, enc, &p.tm_k0, ws_k, a->total_k, hkv, kRope, 1, BN))) return rc;
     if ((rc = make_map(fn, enc, &p.tm_k12, a->k, a->total_k, hkv, kDqk, 1, BN))) return rc;
@@ -392,6 +409,9 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
     r.ring_v = static_cast<const uint16_t*>(a->v_cache);
     r.ws_k = ws_k;
     r.ws_v = ws_v;
+    r.total_q = kind == 0 ? a->total_q : 0;
+    r.cu_q = a->cu_seqlens_q;
+    r.cs_q = cs_q;
     r.rope = p.rope;
     r.status = d.status;
     cudaError_t e = launch_rope_k(r, st);

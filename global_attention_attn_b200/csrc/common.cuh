@@ -67,4 +67,43 @@ __device__ __forceinline__ void rope_chunk_pair_cs(uint4& lo, uint4& hi, const f
   }
 }
 
+// Same rotation on packed fp32 pairs: cs[w] = (cos_a, sin_a, cos_b, sin_b) for the
+// two frequencies held by 32-bit word w of the chunks.
+__device__ __forceinline__ void rope_chunk_pair_cs4(uint4& lo, uint4& hi, const float4* cs) {
+  uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float4 t = cs[w];
+    // x = (x0, x1), y = (y0, y1), c = (c0, c1), s = (s0, s1)
+    uint64_t x, y, c, sn, ns, r0, r1;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(a[w] << 16), "r"(a[w] & 0xFFFF0000u));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "r"(b[w] << 16), "r"(b[w] & 0xFFFF0000u));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(t.x), "f"(t.z));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(sn) : "f"(t.y), "f"(t.w));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ns) : "f"(-t.y), "f"(-t.w));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r0) : "l"(y), "l"(ns));      // -y s
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(r0) : "l"(x), "l"(c));   // x c - y s
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r1) : "l"(x), "l"(sn));      // x s
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(r1) : "l"(y), "l"(c));   // y c + x s
+    float a0, a1, b0, b1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(r0));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(r1));
+    a[w] = pack2_f16(a0, a1);
+    b[w] = pack2_f16(b0, b1);
+  }
+}
+
+// Same angle, reduced in float64, with the MUFU sine / cosine of the reduced
+// float32 angle (absolute error ~1e-6 on [-pi, pi], far below the fp16 rounding
+// of the rotated values).  For per-tile tables where the accurate sincosf costs
+// more than the whole rotation.
+__device__ __forceinline__ void rope_cos_sin_fast(int pos, double inv_freq, float* c, float* s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double theta = double(pos) * inv_freq;
+  const double k = rint(theta * (1.0 / two_pi));
+  const float r = float(fma(-k, two_pi, theta));
+  __sincosf(r, s, c);
+}
+
 }  // namespace mimo

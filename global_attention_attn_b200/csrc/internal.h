@@ -69,6 +69,7 @@ struct PrefillParams {
   CUtensorMap tm_k0;   // key dims 0..63 source, box {64, 1, BN}
   CUtensorMap tm_k12;  // key dims 64..191 source (x = 64, 128), box {64, 1, BN}
   CUtensorMap tm_v;    // value source (x = 0, 64), box {64, 1, BN}
+  CUtensorMap tm_cs;   // per-query-row cos/sin table [total_q, 64] fp32, box {64, 16} (sliding window)
   int num_seqs, total_q, hkv, mode, window;
   int seq_base;  // index of this launch's first sequence in the whole batch (launches take <= 256)
   const int32_t* cu_q;
@@ -96,6 +97,11 @@ struct RopeKParams {
   const uint16_t* ring_v;
   uint16_t* ws_k;  // contig: [total_k, hkv, 64]; ext: [total_k + 128*B, hkv, 192]
   uint16_t* ws_v;  // ext: [total_k + 128*B, hkv, 128]
+  // per-query-row (cos, sin) of the 32 rotary frequencies, or null
+  int total_q;
+  const int32_t* cu_q;
+  float2* cs_q;    // [total_q, 32]
+  int key_blocks;  // blocks of the launch that work on keys; the rest fill cs_q
   RopeFreqs rope;
   unsigned* status;
 };

@@ -46,8 +46,8 @@ constexpr int kThreads = 192;
 template <int KIND>
 struct Cfg;
 template <>
-struct Cfg<0> {  // sliding window
-  static constexpr int G = 8, R = 16, BN = 144, NQ = 2, NK = 1, NV = 1;
+struct Cfg<0> {  // sliding window (prefill_swa_kernel)
+  static constexpr int G = 8, R = 16, BN = 144;
 };
 template <>
 struct Cfg<1> {  // global (or any window wider than 129)
@@ -482,7 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 #pragma unroll
         for (int c = 0; c + 32 <= BN; c += 32) tmem_ld32(t_lane + b * kColS1 + c, sr + c);
         if (BN % 32) tmem_ld16(t_lane + b * kColS1 + (BN / 32) * 32, sr + (BN / 32) * 32);
-        tmem_wait_ld();
+        static_assert(BN == 128, "the wait below binds 128 registers");
+        tmem_wait_ld_r64(sr);
+        tmem_wait_ld_r64(sr + 64);
         float* sv = reinterpret_cast<float*>(sr);
         const int kt0 = key_tile_start<KIND>(T, j_lo + j);
         const bool interior = kt0 >= T.key_lo && kt0 + BN - 1 <= T.qpos0 &&
@@ -514,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           for (int c = 0; c < 128; c += 32) {
             uint32_t o[32];
             tmem_ld32(t_lane + kColO + c, o);
-            tmem_wait_ld();
+            tmem_wait_ld_r32(o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st16(t_lane + kColO + c, o);
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       for (int c = 0; c < 128; c += 32) {
         uint32_t o[32];
         tmem_ld32(t_lane + kColO + c, o);
-        tmem_wait_ld();
+        tmem_wait_ld_r32(o);
         uint4 pk[4];
         uint32_t* w32 = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
@@ -587,12 +589,490 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   }
 }
 
+// ---------------------------------------------------------------- sliding window
+// The sliding-window layer (window <= 129) has exactly one 144-key tile per M
+// tile, so there is no loop over key tiles to pipeline.  Instead two softmax
+// warpgroups take alternate M tiles (WG0 the even ones, WG1 the odd ones) and
+// work on them at the same time.  Each tile owns a 256-column TMEM region:
+// S in columns 0..143, then P (bf16 pairs) over columns 0..71 and O in columns
+// 72..199, which only holds S values the softmax has already read.  Warps 10
+// and 11 apply the partial RoPE to each Q tile in shared memory, with a
+// per-row (cos, sin) table that the key pre-pass computes once per query row.  With 12
+// warps, each SM sub-partition holds 3, which caps registers at 168 per
+// thread; the softmax therefore reads S in 48-column chunks, twice (row
+// maximum, then exponentials).  The MMA
+// lane issues QK^T of tile t before PV of tile t-1; QK^T of tile t waits until
+// the epilogue of tile t-2 (same region) has read O.
+namespace {
+struct SwaLayout {
+  using C = Cfg<0>;
+  static constexpr int kQChunk = 128 * 128;
+  static constexpr int kQStage = 3 * kQChunk;
+  static constexpr int kKChunk = C::BN * 128;
+  static constexpr int kVChunk = C::BN * 128;
+  static constexpr int kOffQ = 0;                          // 2 stages
+  static constexpr int kOffK = kOffQ + 2 * kQStage;         // 1 stage, 3 chunks
+  static constexpr int kOffV = kOffK + 3 * kKChunk;         // 1 stage, 2 chunks
+  static constexpr int kOffBar = kOffV + 2 * kVChunk;
+  static constexpr int kNumBars = 24;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffSeq = kOffMisc + 16;
+  static constexpr int kOffSink = kOffSeq + 6 * (kMaxSeqs + 1) * 4;
+  static constexpr int kOffCS = (kOffSink + 64 * 4 + 1023) / 1024 * 1024;  // float2 [2][R][32] per Q stage (TMA)
+  static constexpr int kCSStage = C::R * 32 * 8;
+  static constexpr int kBytes = kOffCS + 2 * kCSStage;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(kOffCS % 128 == 0 && kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
+                "TMA destinations: 1024-byte aligned for 128-byte swizzle, 128-byte otherwise");
+};
+constexpr int kSwaThreads = 384;
+constexpr uint32_t kSwaRegion = 256;  // TMEM columns per tile region
+constexpr uint32_t kSwaColO = 72;     // O inside a region
+}  // namespace
+
+__global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __grid_constant__ PrefillParams p) {
+  using C = Cfg<0>;
+  using Ly = SwaLayout;
+  constexpr int G = C::G, R = C::R, BN = C::BN;
+  constexpr int CH = BN / 3;  // 48 columns per softmax chunk
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = sbase + Ly::kOffBar;
+  auto q_full = [&](int b) { return bar0 + 8 * (0 + b); };
+  auto q_rot = [&](int b) { return bar0 + 8 * (2 + b); };
+  auto q_empty = [&](int b) { return bar0 + 8 * (4 + b); };
+  const uint32_t k_full = bar0 + 8 * 6, k_empty = bar0 + 8 * 7, v_full = bar0 + 8 * 8, v_empty = bar0 + 8 * 9;
+  auto s_full = [&](int b) { return bar0 + 8 * (10 + b); };
+  auto p_full = [&](int b) { return bar0 + 8 * (12 + b); };
+  auto pv_done = [&](int b) { return bar0 + 8 * (14 + b); };
+  auto o_empty = [&](int b) { return bar0 + 8 * (16 + b); };
+  const uint32_t drain = bar0 + 8 * 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::kOffMisc + 4);
+  const SeqTable S = seq_table(smem + Ly::kOffSeq);
+  float* sink_l2 = reinterpret_cast<float*>(smem + Ly::kOffSink);
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full(b), 1);
+      mbar_init(q_rot(b), 64);
+      mbar_init(q_empty(b), 1);
+      mbar_init(s_full(b), 1);
+      mbar_init(p_full(b), 128);
+      mbar_init(pv_done(b), 1);
+      mbar_init(o_empty(b), 128);
+    }
+
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) fill_seq_table<0>(p, S);
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x >= 64 && threadIdx.x < 128)
+    sink_l2[threadIdx.x - 64] = p.sink ? p.sink[threadIdx.x - 64] * kLog2e : -INFINITY;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  unsigned* status = p.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producers (Q, K, V lanes)
+    if (lane < 3) {
+      if (lane == 0) {
+        tma_prefetch(&p.tm_q);
+        tma_prefetch(&p.tm_k0);
+        tma_prefetch(&p.tm_k12);
+        tma_prefetch(&p.tm_v);
+        tma_prefetch(&p.tm_cs);
+      }
+      bool ok = true;
+      int mt = 0;
+      for (int w = blockIdx.x; ok; w += gridDim.x, ++mt) {
+        TileInfo T;
+        if (!locate<0>(p, S, w, T)) break;
+        const int row = T.krow_base + (T.qpos0 - 128 - T.kpos_base);
+        if (lane == 0) {
+          const int b = mt & 1;
+          if (mt >= 2 && !(ok = mbar_wait(q_empty(b), ((mt >> 1) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)))
+            break;
+          const uint32_t qdst = sbase + Ly::kOffQ + b * Ly::kQStage;
+          mbar_expect_tx(q_full(b), Ly::kQStage + Ly::kCSStage);
+          for (int c = 0; c < 3; ++c)
+            tma_load_3d(qdst + c * Ly::kQChunk, &p.tm_q, q_full(b), 64 * c, T.g * G, T.q_row0);
+          tma_load_2d(sbase + Ly::kOffCS + b * Ly::kCSStage, &p.tm_cs, q_full(b), 0, T.q_row0);
+        } else if (lane == 1) {
+          if (mt >= 1 && !(ok = mbar_wait(k_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          const uint32_t kdst = sbase + Ly::kOffK;
+          mbar_expect_tx(k_full, 3 * Ly::kKChunk);
+          tma_load_3d(kdst, &p.tm_k0, k_full, 0, T.g, row);
+          tma_load_3d(kdst + Ly::kKChunk, &p.tm_k12, k_full, 64, T.g, row);
+          tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full, 128, T.g, row);
+        } else {
+          if (mt >= 1 && !(ok = mbar_wait(v_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          const uint32_t vdst = sbase + Ly::kOffV;
+          mbar_expect_tx(v_full, 2 * Ly::kVChunk);
+          tma_load_3d(vdst, &p.tm_v, v_full, 0, T.g, row);
+          tma_load_3d(vdst + Ly::kVChunk, &p.tm_v, v_full, 64, T.g, row);
+        }
+      }
+      if (!ok) {
+        int dummy = 0;
+        for (int b = 0; b < 2; ++b) mbar_wait(q_full(b), 0, &dummy, nullptr, 0, 50000000ull);
+        mbar_wait(k_full, 0, &dummy, nullptr, 0, 50000000ull);
+        mbar_wait(v_full, 0, &dummy, nullptr, 0, 50000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (lane 0)
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk_rot = idesc_f32acc(128, BN, 0, 0, 0);  // dims 0..63: fp16 x fp16
+      constexpr uint32_t idesc_qk = idesc_f32acc(128, BN, 0, 0, 1);      // dims 64..191: bf16 x bf16
+      constexpr uint32_t idesc_pv = idesc_f32acc(128, 128, 0, 1, 1);
+      bool ok = true;
+      auto issue_pv = [&](int t) -> bool {
+        const int b = t & 1;
+        if (!mbar_wait(p_full(b), (t >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        if (!mbar_wait(v_full, t & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        tc_fence_after();
+        const uint32_t reg = tmem + b * kSwaRegion;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(sbase + Ly::kOffV + kk * 2048, Ly::kVChunk, 1024);
+          tc_mma_ts(reg + kSwaColO, reg + kk * 8, bd, idesc_pv, kk == 0 ? 0u : 1u);
+        }
+        tc_commit(v_empty);
+        tc_commit(pv_done(b));
+        return true;
+      };
+      // Two cursors: tq = next tile to multiply QK^T for, tp = next tile to multiply PV
+      // for (tp <= tq <= tp + 1: two TMEM regions).  Whichever is ready goes first, so
+      // one warpgroup's PV never waits on the other warpgroup's next Q.
+      auto issue_qk = [&](int t) {
+        const int b = t & 1;
+        tc_fence_after();
+        const uint32_t qbase = sbase + Ly::kOffQ + b * Ly::kQStage;
+        const uint32_t kbase = sbase + Ly::kOffK;
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sdesc_sw128(qbase + c * Ly::kQChunk + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kbase + c * Ly::kKChunk + kk * 32, 16, 1024);
+            tc_mma_ss(tmem + b * kSwaRegion, ad, bd, c == 0 ? idesc_qk_rot : idesc_qk, (c | kk) ? 1u : 0u);
+          }
+        tc_commit(s_full(b));
+        tc_commit(k_empty);
+        tc_commit(q_empty(b));
+      };
+      int tq = 0, tp = 0;
+      bool have_q;
+      {
+        TileInfo T;
+        have_q = locate<0>(p, S, blockIdx.x, T);
+      }
+      uint64_t t_last = global_timer_ns();
+      while (have_q || tp < tq) {
+        bool progress = false;
+        if (tp < tq) {
+          const int b = tp & 1;
+          if (mbar_test_wait(p_full(b), (tp >> 1) & 1) && mbar_test_wait(v_full, tp & 1)) {
+            ok = issue_pv(tp);  // its waits succeed at once
+            if (!ok) break;
+            ++tp;
+            progress = true;
+          }
+        }
+        if (have_q && tq <= tp + 1) {
+          const int b = tq & 1;
+          if (mbar_test_wait(q_rot(b), (tq >> 1) & 1) && mbar_test_wait(k_full, tq & 1) &&
+              (tq < 2 || mbar_test_wait(o_empty(b), ((tq >> 1) - 1) & 1))) {
+            issue_qk(tq);
+            ++tq;
+            TileInfo T;
+            have_q = locate<0>(p, S, blockIdx.x + tq * gridDim.x, T);
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = global_timer_ns();
+        } else if (!*abort_flag && global_timer_ns() - t_last <= 2000000000ull) {
+          __nanosleep(32);  // yield the issue slots this sub-partition shares with softmax warps
+        } else if (*abort_flag) {
+          ok = false;
+          break;
+        } else if (global_timer_ns() - t_last > 2000000000ull) {
+          *abort_flag = 1;
+          atomicOr(status, MIMO_STATUS_TIMEOUT);
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) {
+        int dummy = 0;
+        tc_commit(drain);
+        mbar_wait(drain, 0, &dummy, nullptr, 0, 50000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ Q RoPE (warps 10, 11)
+    // Dims 0..63 of the tile's 128 rows are rotated in place (128-byte swizzled rows)
+    // to fp16 with the (cos, sin) rows the producer loaded next to the Q tile.
+    const int lt = threadIdx.x - 320;  // 0..63
+    bool ok = true;
+    for (int mt = 0, w = blockIdx.x; ok; ++mt, w += gridDim.x) {
+      TileInfo T;
+      if (!locate<0>(p, S, w, T)) break;
+      const int b = mt & 1;
+      if (!(ok = mbar_wait(q_full(b), (mt >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+      const float4* cs = reinterpret_cast<const float4*>(smem + Ly::kOffCS + b * Ly::kCSStage);
+      uint8_t* qs = smem + Ly::kOffQ + b * Ly::kQStage;
+      // work item k: head h = k & 7, chunk pair u = (k >> 3) & 3, position r = k >> 5 (row 8r + h):
+      // the 8 lanes of a shared-memory phase hit 8 distinct swizzled 16-byte groups of Q and
+      // read one broadcast (cos, sin) address.
+#pragma unroll 2
+      for (int i = 0; i < 128 * 4 / 64; ++i) {
+        const int k = lt + 64 * i;
+        const int m = ((k >> 5) << 3) + (k & 7), u = (k >> 3) & 3, sw = m & 7;
+        uint8_t* row = qs + m * 128;
+        uint4* plo = reinterpret_cast<uint4*>(row + ((u ^ sw) << 4));
+        uint4* phi = reinterpret_cast<uint4*>(row + (((u + 4) ^ sw) << 4));
+        uint4 lo = *plo, hi = *phi;
+        // (cos, sin) of frequencies 8u..8u+7 at the row's position: 4 x float4
+        rope_chunk_pair_cs4(lo, hi, cs + (m / G) * 16 + 4 * u);
+        *plo = lo;
+        *phi = hi;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_rot(b));
+    }
+  } else {
+    // ------------------------------------------------------------ two softmax warpgroups
+    const int wg = (warp - 2) >> 2;        // 0: warps 2..5, 1: warps 6..9
+    const int quad = warp & 3;
+    const int m = quad * 32 + lane;        // TMEM lane = M row
+    const int r = m / G, hq = m % G;
+    const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16) + wg * kSwaRegion;
+    const float c_log2 = p.scale_log2;
+    auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
+    };
+    for (int mt = wg, w = blockIdx.x + wg * gridDim.x;; mt += 2, w += 2 * gridDim.x) {
+      TileInfo T;
+      if (!locate<0>(p, S, w, T)) break;
+      const int b = wg;  // == mt & 1
+      const uint32_t ph = (mt >> 1) & 1;
+      // ---- softmax over the 144-key tile, two passes of 72 columns
+      const bool row_valid = r < T.rows_valid;
+      const int qp = T.qpos0 + r;
+      const int head = T.g * G + hq;
+      const int kt0 = T.qpos0 - 128;
+      const int vis_hi = row_valid ? qp : -0x40000000;
+      const int vis_lo = max(T.key_lo, qp - p.window + 1);
+      const int ca = vis_lo - kt0, ce = vis_hi - kt0;  // visible columns [ca, ce]
+      if (!wait_w(s_full(b), ph)) break;
+      tc_fence_after();
+      // Columns 16..127 of the tile are visible to all 16 positions whenever the whole
+      // window exists (ca <= 16, ce >= 127 for every row): only the 16 edge columns
+      // on each side need the per-element mask then.
+      const bool band = __all_sync(0xffffffffu, ca <= 16 && ce >= 127);
+      const float sink = sink_l2[head];
+      float m_use, la[4];
+      if (band) {
+        // Columns 16..127 are visible to every row.  S is read in chunks of 32 columns
+        // (the last one 16): the edge columns are the first half of chunk 0 and all of
+        // chunk 4, chunks 1..3 need no mask.  Each chunk's TMEM load is issued before
+        // the previous chunk is processed (two register buffers).
+        uint32_t buf[2][32];
+        float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        auto ld = [&](int h, uint32_t* d) {
+          if (h < 4) tmem_ld32(t_lane + 32 * h, d);
+          else tmem_ld16(t_lane + 128, d);
+        };
+        auto edge_col = [&](int h, int c) { return (h == 0 && c < 16) || h == 4; };
+        auto max_chunk = [&](const uint32_t* sr, int h) {
+#pragma unroll
+          for (int c = 0; c < (h < 4 ? 32 : 16); ++c) {
+            const int cc = 32 * h + c;
+            if (!edge_col(h, c) || (cc >= ca && cc <= ce)) mxa[c & 3] = fmaxf(mxa[c & 3], __uint_as_float(sr[c]));
+          }
+        };
+        ld(0, buf[0]);
+        tmem_wait_ld_r32(buf[0]);
+#pragma unroll
+        for (int h = 0; h < 5; ++h) {
+          if (h < 4) ld(h + 1, buf[(h + 1) & 1]);
+          else ld(0, buf[1]);  // chunk 0 again, for the exponentials
+          max_chunk(buf[h & 1], h);
+          if (h == 3) tmem_wait_ld_r16_after(buf[0], mxa[0], mxa[1], mxa[2], mxa[3]);
+          else tmem_wait_ld_r32_after(buf[(h + 1) & 1], mxa[0], mxa[1], mxa[2], mxa[3]);
+        }
+        const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+        const float m_row = fmaxf(sink, mx * c_log2);
+        m_use = m_row == -INFINITY ? 0.f : m_row;
+        uint64_t la2 = pack_f32x2(p.sink ? ex2(sink - m_use) : 0.f, 0.f);
+        const uint64_t cl2 = pack_f32x2(c_log2, c_log2), nm2 = pack_f32x2(-m_use, -m_use);
+        auto exp_chunk = [&](const uint32_t* sr, int h) {
+#pragma unroll
+          for (int g = 0; g < (h < 4 ? 32 : 16); g += 16) {  // 16 columns -> 8 packed words -> one TMEM store
+            uint32_t pk[8];
+#pragma unroll
+            for (int c = g; c < g + 16; c += 2) {
+              const uint64_t t = fma_f32x2(pack_f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, nm2);
+              float p0 = ex2(lo_f32(t)), p1 = ex2(hi_f32(t));
+              if (edge_col(h, c)) {
+                const int cc = 32 * h + c;
+                p0 = (cc >= ca && cc <= ce) ? p0 : 0.f;
+                p1 = (cc + 1 >= ca && cc + 1 <= ce) ? p1 : 0.f;
+              }
+              la2 = add_f32x2(la2, pack_f32x2(p0, p1));
+              pk[(c - g) / 2] = pack_bf16x2(p0, p1);
+            }
+            tmem_st8(t_lane + (32 * h + g) / 2, pk);
+          }
+        };
+        // chunk 0 is in buf[1]
+#pragma unroll
+        for (int h = 0; h < 5; ++h) {
+          if (h < 4) ld(h + 1, buf[h & 1]);
+          exp_chunk(buf[(h + 1) & 1], h);
+          if (h == 3) tmem_wait_ld_r16_after(buf[h & 1], la2);
+          else if (h < 3) tmem_wait_ld_r32_after(buf[h & 1], la2);
+        }
+        la[0] = lo_f32(la2);
+        la[1] = hi_f32(la2);
+        la[2] = la[3] = 0.f;
+      } else {
+        float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int h = 0; h < 3; ++h) {
+          uint32_t sr[CH];
+          tmem_ld32(t_lane + h * CH, sr);
+          tmem_ld16(t_lane + h * CH + 32, sr + 32);
+          tmem_wait_ld_r32(sr);
+          tmem_wait_ld_r16(sr + 32);
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            const int cc = h * CH + c;
+            if (cc >= ca && cc <= ce) mxa[c & 3] = fmaxf(mxa[c & 3], __uint_as_float(sr[c]));
+          }
+        }
+        const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+        const float m_row = fmaxf(sink, mx * c_log2);
+        m_use = m_row == -INFINITY ? 0.f : m_row;
+        la[0] = p.sink ? ex2(sink - m_use) : 0.f;
+        la[1] = la[2] = la[3] = 0.f;
+#pragma unroll 1
+        for (int h = 0; h < 3; ++h) {
+          uint32_t sr[CH];
+          tmem_ld32(t_lane + h * CH, sr);
+          tmem_ld16(t_lane + h * CH + 32, sr + 32);
+          tmem_wait_ld_r32(sr);
+          tmem_wait_ld_r16(sr + 32);
+          uint32_t pk[CH / 2];
+#pragma unroll
+          for (int c = 0; c < CH; c += 2) {
+            const int cc = h * CH + c;
+            float p0 = ex2(fmaf(__uint_as_float(sr[c]), c_log2, -m_use));
+            float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), c_log2, -m_use));
+            p0 = (cc >= ca && cc <= ce) ? p0 : 0.f;
+            p1 = (cc + 1 >= ca && cc + 1 <= ce) ? p1 : 0.f;
+            la[(c >> 1) & 3] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(t_lane + h * (CH / 2), pk);
+          tmem_st8(t_lane + h * (CH / 2) + 16, pk + 16);
+        }
+      }
+      const float l_row = (la[0] + la[1]) + (la[2] + la[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(b));
+      // ---- epilogue: O * v_scale / l -> bf16, LSE
+      if (!wait_w(pv_done(b), ph)) break;
+      tc_fence_after();
+      const float sc = p.v_scale / l_row;
+      uint16_t* orow = p.out + (long(T.q_row0 + r) * kHq + head) * kDv;
+      {
+        const uint64_t sc2 = pack_f32x2(sc, sc);
+        uint32_t oa[32], ob[32];
+        auto store_chunk = [&](uint32_t* o, int c) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t t = mul_f32x2(pack_f32x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), sc2);
+            o[i] = pack_bf16x2(lo_f32(t), hi_f32(t));
+          }
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+        };
+        tmem_ld32(t_lane + kSwaColO, oa);
+        tmem_wait_ld_r32(oa);
+        tmem_ld32(t_lane + kSwaColO + 32, ob);
+        store_chunk(oa, 0);
+        tmem_wait_ld_r32(ob);
+        tmem_ld32(t_lane + kSwaColO + 64, oa);
+        store_chunk(ob, 32);
+        tmem_wait_ld_r32(oa);
+        tmem_ld32(t_lane + kSwaColO + 96, ob);
+        store_chunk(oa, 64);
+        tmem_wait_ld_r32(ob);
+        store_chunk(ob, 96);
+      }
+      if (row_valid && p.lse) p.lse[long(T.q_row0 + r) * kHq + head] = (m_use + __log2f(l_row)) * kLn2;
+      tc_fence_before();
+      mbar_arrive(o_empty(b));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- key pre-pass
 // contig: 4 lanes per (row, kv head) write rotated dims 0..63 (fp16) into ws_k.
 // ext: one warp per (ext row, kv head) writes the full rotated key (dims 0..63
 //      fp16, 64..191 bf16) and the value: halo rows copied from the ring (which
 //      stores the same format), new rows rotated from k / v.
 __global__ void __launch_bounds__(256) rope_k_kernel(const RopeKParams p) {
+  if (int(blockIdx.x) >= p.key_blocks) {
+    // (cos, sin) of the 32 rotary frequencies at each query row's position: one warp per row
+    const long row = (long(blockIdx.x - p.key_blocks) * blockDim.x + threadIdx.x) >> 5;
+    const int j = threadIdx.x & 31;
+    if (row >= p.total_q) return;
+    int lo = 0, hi = p.num_seqs;  // sequence of the row
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.cu_q[mid] <= row) lo = mid; else hi = mid;
+    }
+    const int qlen = p.cu_q[lo + 1] - p.cu_q[lo];
+    const int ctx = (p.cache_lens ? p.cache_lens[lo] : 0) + (p.cu_k[lo + 1] - p.cu_k[lo]);
+    const int pos = ctx - qlen + int(row - p.cu_q[lo]);
+    float c, sn;
+    rope_cos_sin(pos, p.rope.inv_freq[j], &c, &sn);
+    p.cs_q[row * kHalf + j] = make_float2(c, sn);
+    return;
+  }
   const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
   if (p.mode == kModeContig) {
     const long item = gt >> 2;
@@ -659,8 +1139,11 @@ cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s) {
   long threads;
   if (p.mode == kModeContig) threads = long(p.total_k) * p.hkv * 4;
   else threads = (long(p.total_k) + 128L * p.num_seqs) * p.hkv * 32;
-  if (threads == 0) return cudaSuccess;
-  rope_k_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(p);
+  RopeKParams q = p;
+  q.key_blocks = int((threads + 255) / 256);
+  const long cs_blocks = q.cs_q ? (long(q.total_q) * 32 + 255) / 256 : 0;
+  if (q.key_blocks + cs_blocks == 0) return cudaSuccess;
+  rope_k_kernel<<<unsigned(q.key_blocks + cs_blocks), 256, 0, s>>>(q);
   return cudaGetLastError();
 }
 
@@ -670,10 +1153,10 @@ int prefill_key_tile(int kind) { return kind == 0 ? Cfg<0>::BN : Cfg<1>::BN; }
 cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
   if (kind == 0) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Layout<0>::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SwaLayout::kAlloc);
     if (e != cudaSuccess) return e;
-    prefill_kernel<0><<<grid, kThreads, Layout<0>::kAlloc, s>>>(p);
+    prefill_swa_kernel<<<grid, kSwaThreads, SwaLayout::kAlloc, s>>>(p);
   } else {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Layout<1>::kAlloc);

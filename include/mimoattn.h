@@ -100,7 +100,8 @@ typedef struct {
  * pre-RoPE; v [total_k, Hkv, 128] bf16; out [total_q, 64, 128] bf16;
  * lse [total_q, 64] fp32 natural-log LSE including the sink (may be NULL).
  * The workspace (size from mimo_attn_prefill_workspace_size) holds rotated
- * key copies; its contents need no initialisation.
+ * key copies and a per-query-row table of the rotary cos / sin values; its
+ * contents need no initialisation.
  * Cache slots at or beyond a sequence's context must hold finite values
  * (e.g. zero-initialise caches): they are read and masked, not skipped.
  */
@@ -128,7 +129,8 @@ typedef struct {
 } mimo_prefill_args;
 
 /* Bytes of workspace mimo_attn_prefill needs for these sizes. */
-MIMO_API size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_k, int num_kv_heads, int cache_kind);
+MIMO_API size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_q, int total_k, int num_kv_heads,
+                                                 int cache_kind);
 
 MIMO_API int mimo_attn_prefill(const mimo_prefill_args* args, void* stream);
 

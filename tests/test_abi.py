@@ -62,10 +62,11 @@ def test_struct_layouts_match_c(tmp_path):
 
 
 def test_workspace_sizes():
-    assert M.prefill_workspace_size(1, 512, 8, M.MIMO_CACHE_NONE) == 512 * 8 * 64 * 2
-    assert M.prefill_workspace_size(3, 100, 4, M.MIMO_CACHE_PAGED) == 0
-    ring = M.prefill_workspace_size(1, 8192, 8, M.MIMO_CACHE_RING)
-    assert ring >= (8192 + 128) * 8 * (192 + 128) * 2
+    # rotated key dims (fp16) + a cos/sin table of 32 float2 per query row
+    assert M.prefill_workspace_size(1, 512, 512, 8, M.MIMO_CACHE_NONE) == 512 * 8 * 64 * 2 + 512 * 32 * 8
+    assert M.prefill_workspace_size(3, 100, 100, 4, M.MIMO_CACHE_PAGED) == 0
+    ring = M.prefill_workspace_size(1, 8192, 8192, 8, M.MIMO_CACHE_RING)
+    assert ring >= (8192 + 128) * 8 * (192 + 128) * 2 + 8192 * 32 * 8
     assert M.decode_workspace_size(64, 128, 8, 128) == 0          # one split: no partials
     ns = (65536 + 511) // 512
     assert M.decode_workspace_size(64, 65536, 4, 0) >= 64 * 64 * ns * (128 + 2) * 4
