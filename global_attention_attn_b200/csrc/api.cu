@@ -122,10 +122,12 @@ int make_map(const char* fn, EncodeTiledFn enc, CUtensorMap* m, const void* base
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Keys per decode split (a multiple of the kernel's 64-key tile).
 int decode_split_len(int max_seq_len, int window) {
   const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
   if (n <= 256) return 256;
-  return 512;
+  if (n <= 8192) return 512;
+  return 1024;
 }
 
 }  // namespace
@@ -242,7 +244,16 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   }
   DevState d;
   if (int rc = dev_state(fn, &d)) return rc;
+  EncodeTiledFn enc;
+  if (int rc = get_encoder(fn, &enc)) return rc;
   DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  {
+    const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * kPage : long(a->num_pages) * kPage;
+    int rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 64);
+    if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 64);
+    if (rc) return rc;
+  }
   p.batch = a->batch;
   p.hkv = a->layer.num_kv_heads;
   p.group = kHq / p.hkv;
@@ -269,7 +280,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
                  : nullptr;
   p.rope = make_freqs(a->layer.rope_base);
   p.status = d.status;
-  cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_decode(p, d.sms, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return MIMO_OK;
 }

@@ -68,7 +68,7 @@ def test_workspace_sizes():
     ring = M.prefill_workspace_size(1, 8192, 8192, 8, M.MIMO_CACHE_RING)
     assert ring >= (8192 + 128) * 8 * (192 + 128) * 2 + 8192 * 32 * 8
     assert M.decode_workspace_size(64, 128, 8, 128) == 0          # one split: no partials
-    ns = (65536 + 511) // 512
+    ns = (65536 + 1023) // 1024                                   # 1024-key splits past 8192 keys
     assert M.decode_workspace_size(64, 65536, 4, 0) >= 64 * 64 * ns * (128 + 2) * 4
 
 
