@@ -53,14 +53,15 @@ class MimoPrefillArgs(C.Structure):
                 ("q", _P), ("k", _P), ("v", _P), ("cu_seqlens_q", _P), ("cu_seqlens_k", _P), ("cache_lens", _P),
                 ("cache_kind", C.c_int), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
                 ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P), ("workspace", _P),
-                ("workspace_bytes", C.c_size_t)]
+                ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P), ("ev_kernel_end", _P)]
 
 
 class MimoDecodeArgs(C.Structure):
     _fields_ = [("layer", MimoLayer), ("batch", C.c_int), ("max_seq_len", C.c_int), ("q", _P),
                 ("seq_lens", _P), ("cache_kind", C.c_int), ("k_cache", _P), ("v_cache", _P),
                 ("block_table", _P), ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P),
-                ("workspace", _P), ("workspace_bytes", C.c_size_t)]
+                ("workspace", _P), ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P),
+                ("ev_kernel_end", _P)]
 
 
 class MimoAppendArgs(C.Structure):
@@ -144,13 +145,24 @@ def decode_workspace_size(batch: int, max_seq_len: int, num_kv_heads: int, windo
     return int(lib().mimo_attn_decode_workspace_size(batch, max_seq_len, num_kv_heads, window))
 
 
+def _events(pair):
+    """cudaEvent_t handles of a (begin, end) pair of torch.cuda.Event (None: no hooks)."""
+    if pair is None:
+        return None, None
+    handles = [int(ev.cuda_event) for ev in pair]
+    if len(handles) != 2 or not all(handles):
+        raise ValueError("kernel_events: pass two torch.cuda.Event that have been recorded once")
+    return handles[0], handles[1]
+
+
 def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int, rope_base: float, window: int,
                       sink=None, cache_lens=None, cache_kind: int = MIMO_CACHE_NONE, k_cache=None, v_cache=None,
                       block_table=None, num_pages: int = 0, out=None, lse=None, workspace=None,
                       softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None,
-                      with_lse: bool = True):
+                      with_lse: bool = True, kernel_events=None):
     """Varlen prefill (see include/mimoattn.h).  Tensors are CUDA tensors: q/k/v/caches bf16,
-    index tensors int32, sink fp32.  Returns (out, lse)."""
+    index tensors int32, sink fp32.  kernel_events: optional (begin, end) pair of recorded-once
+    torch.cuda.Event placed around the attention kernel.  Returns (out, lse)."""
     import torch
     total_q = q.shape[0]
     num_seqs = cu_seqlens_q.shape[0] - 1
@@ -174,6 +186,7 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
     a.out, a.lse = _ptr(out), _ptr(lse)
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
     _check(lib().mimo_attn_prefill(C.byref(a), _stream(stream)))
     return out, lse
 
@@ -181,8 +194,9 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
 def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_base: float, window: int,
                      cache_kind: int, k_cache, v_cache, block_table=None, num_pages: int = 0, sink=None, out=None,
                      lse=None, workspace=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE,
-                     stream=None, with_lse: bool = True):
-    """Decode step (see include/mimoattn.h).  Returns (out, lse)."""
+                     stream=None, with_lse: bool = True, kernel_events=None):
+    """Decode step (see include/mimoattn.h).  kernel_events as for mimo_attn_prefill (around the
+    split kernel, not the combine).  Returns (out, lse)."""
     import torch
     B = q.shape[0]
     if out is None:
@@ -203,6 +217,7 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
     a.out, a.lse = _ptr(out), _ptr(lse)
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
     _check(lib().mimo_attn_decode(C.byref(a), _stream(stream)))
     return out, lse
 

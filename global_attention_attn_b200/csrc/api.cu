@@ -122,7 +122,7 @@ int make_map(const char* fn, EncodeTiledFn enc, CUtensorMap* m, const void* base
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Keys per decode split (a multiple of the kernel's 64-key tile).
+// Keys per decode split (a multiple of the kernel's 16-key tile).
 int decode_split_len(int max_seq_len, int window) {
   const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
   if (n <= 256) return 256;
@@ -250,8 +250,9 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   std::memset(&p, 0, sizeof(p));
   {
     const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * kPage : long(a->num_pages) * kPage;
-    int rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 64);
-    if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 64);
+    int rc = make_map(fn, enc, &p.tm_q, a->q, a->batch, kHq, kDqk, 16, 1);
+    if (!rc) rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 16);
+    if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 16);
     if (rc) return rc;
   }
   p.batch = a->batch;
@@ -280,7 +281,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
                  : nullptr;
   p.rope = make_freqs(a->layer.rope_base);
   p.status = d.status;
-  cudaError_t e = launch_decode(p, d.sms, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_decode(p, d.sms, static_cast<cudaStream_t>(stream), a->ev_kernel_begin, a->ev_kernel_end);
   if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   return MIMO_OK;
 }
@@ -432,6 +433,10 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   const long work = (long(a->total_q) / R + a->num_seqs + 1) * hkv;
   const int grid = int(work < d.sms ? work : d.sms);
   // one launch per group of at most 256 sequences (the kernel keeps a per-sequence table in shared memory)
+  if (a->ev_kernel_begin) {
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_kernel_begin), st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: ev_kernel_begin: %s", fn, cudaGetErrorString(e));
+  }
   for (int s0 = 0; s0 < a->num_seqs; s0 += kPrefillMaxSeqsPerLaunch) {
     PrefillParams q = p;
     q.seq_base = s0;
@@ -442,6 +447,10 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
     q.block_table = a->block_table ? a->block_table + long(s0) * a->max_pages : nullptr;
     cudaError_t e = launch_prefill(q, kind, grid, st);
     if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  if (a->ev_kernel_end) {
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_kernel_end), st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: ev_kernel_end: %s", fn, cudaGetErrorString(e));
   }
   return MIMO_OK;
 }

@@ -8,13 +8,20 @@
 // per KV head on global layers, 8 on sliding layers, padded to 16).  The sink
 // logit ("Learnable attention sink") joins the final denominator only.
 //
-// Persistent kernel: one CTA per SM walks work units (split, sequence, KV head).
-// Warp 0 streams 64-key K/V tiles with TMA (128-byte swizzle, 4 stages of 40 KB,
-// page ids fetched once per unit); warps 1..4 each take 16 keys of every tile.
-// Each compute warp builds its query fragments straight from global memory and
-// applies the partial RoPE in registers (dims j and j+32 land in the same
-// thread).  A ring cache is read in slot order with each slot's position
-// recovered from the context length: attention does not depend on key order.
+// Work unit = (split, sequence, KV head).  A CTA holds four independent
+// producer / consumer warp pairs, each walking its own units:
+//   producer warp: reads the context length and page ids of the next unit,
+//     computes the unit's rotary cos / sin row (float64 angle), TMA-loads the
+//     unit's 16 query heads into a double-buffered tile, then streams the
+//     unit's keys and values as 16-key TMA tiles (128-byte swizzle) through a
+//     4-stage ring;
+//   consumer warp: builds the query fragments from shared memory with
+//     ldmatrix, rotates dims 0..63 in registers, then runs QK^T, the online
+//     softmax and PV over the tiles with mma.sync, and writes the unit's
+//     result (the final output when a sequence has one split, else partials).
+// No cross-warp merge: one warp owns a unit from its first key to its output.
+// A ring cache is read in slot order with each slot's position recovered from
+// the context length: attention does not depend on key order.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -25,15 +32,23 @@ namespace mimo {
 
 namespace {
 
-constexpr int kTile = 64;  // keys per TMA tile
+constexpr int kPairs = 4;                      // producer / consumer warp pairs per CTA
+constexpr int kThreads = 2 * kPairs * 32;      // warps 0..3 produce, 4..7 consume
+constexpr int kTileK = 16;                     // keys per TMA tile
 constexpr int kStages = 4;
-constexpr int kThreads = 160;
-constexpr int kKChunk = kTile * 128;                    // 64 keys x 64 dims, 2-byte elements
-constexpr int kStageBytes = 3 * kKChunk + 2 * kKChunk;  // K (3 chunks) + V (2 chunks)
-constexpr int kOffMerge = kStages * kStageBytes;
-constexpr int kMergeBytes = 4 * 16 * 4 * 2 + 4 * 16 * kDv * 4;
-constexpr int kOffBar = kOffMerge + kMergeBytes;
-constexpr int kSmemBytes = kOffBar + 16 * 8 + 1024;
+constexpr int kChunk = kTileK * 128;           // 16 keys x 64 dims x 2 bytes
+constexpr int kStageBytes = 5 * kChunk;        // K (3 chunks of 64 dims) + V (2 chunks)
+constexpr int kQChunk = 16 * 128;              // 16 heads x 64 dims x 2 bytes
+constexpr int kQBytes = 3 * kQChunk;
+constexpr int kPairBytes = kStages * kStageBytes + 2 * kQBytes;
+constexpr int kInfoBytes = 32 + 32 * 8;        // unit fields + 32 (cos, sin) pairs
+constexpr int kOffInfo = kPairs * kPairBytes;
+constexpr int kOffBar = kOffInfo + kPairs * 2 * kInfoBytes;
+constexpr int kBarsPerPair = 2 * kStages + 4;  // full, empty, q_full[2], q_empty[2]
+constexpr int kOffTbl = kOffBar + kPairs * kBarsPerPair * 8 + 16;
+constexpr int kMaxTable = 1024;                // sequences of the ordered split enumeration
+constexpr int kSmemBytes = kOffTbl + 2 * (kMaxTable + 1) * 4 + 1024;
+static_assert(kPairBytes % 1024 == 0 && kStageBytes % 1024 == 0 && kQBytes % 1024 == 0, "swizzle alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -64,14 +79,13 @@ __device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-struct Unit {
-  int s, g, split;
-  int ctx, k_begin, k_end;  // keys [k_begin, k_end) of this split
-  int t0, nt;               // tiles (absolute 64-key tiles, or the two ring halves)
+// Unit fields the producer hands to its consumer with the query tile.
+struct UnitInfo {
+  int s, g, split, ctx, k_begin, k_end, t0, nt;  // nt < 0: no more units
 };
 
 // Work unit u of the dense space [split][sequence][kv head]; false if it has no keys.
-__device__ __forceinline__ bool unit_at(const DecodeParams& p, int u, Unit& U) {
+__device__ __forceinline__ bool unit_at(const DecodeParams& p, int u, UnitInfo& U) {
   const int per_split = p.batch * p.hkv;
   U.split = u / per_split;
   const int rem = u - U.split * per_split;
@@ -85,12 +99,54 @@ __device__ __forceinline__ bool unit_at(const DecodeParams& p, int u, Unit& U) {
   U.k_end = min(U.k_begin + p.split_len, U.ctx);
   if (p.cache_kind == MIMO_CACHE_RING) {
     U.t0 = 0;
-    U.nt = 2;  // the 128 slots, in slot order
+    U.nt = kPage / kTileK;  // the 128 slots, in slot order
   } else {
-    U.t0 = U.k_begin / kTile;
-    U.nt = (U.k_end - 1) / kTile - U.t0 + 1;
+    U.t0 = U.k_begin / kTileK;
+    U.nt = (U.k_end - 1) / kTileK - U.t0 + 1;
   }
   return true;
+}
+
+// Keys of sequence s the decode attends (the window's, or the whole context).
+__device__ __forceinline__ int seq_keys(const DecodeParams& p, int ctx) {
+  if (ctx < 1) return 0;
+  return p.window > 0 ? min(ctx, p.window) : ctx;
+}
+
+// Largest s in [0, n) with tbl[s] <= x, for a prefix table with tbl[0] = 0 <= x < tbl[n].
+__device__ __forceinline__ int find_seq(const int* tbl, int n, int x) {
+  int lo = 0, hi = n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tbl[mid] <= x) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Unit v of the ordered enumeration: first every full split (split_len keys) of every
+// sequence, then the shorter last splits, so that a round-robin deal over the warp
+// pairs gives each pair the same number of full units.  tbl_full / tbl_part are
+// prefix sums over sequences of the full-split count and of "has a shorter last split".
+__device__ __forceinline__ void unit_ordered(const DecodeParams& p, const int* tbl_full, const int* tbl_part, int v,
+                                             UnitInfo& U) {
+  int x = v / p.hkv;
+  U.g = v - x * p.hkv;
+  const int F = tbl_full[p.batch];
+  if (x < F) {
+    U.s = find_seq(tbl_full, p.batch, x);
+    U.split = x - tbl_full[U.s];
+  } else {
+    x -= F;
+    U.s = find_seq(tbl_part, p.batch, x);
+    U.split = tbl_full[U.s + 1] - tbl_full[U.s];
+  }
+  U.ctx = p.seq_lens[U.s];
+  const int lo = p.window > 0 ? max(0, U.ctx - p.window) : 0;
+  U.k_begin = lo + U.split * p.split_len;
+  U.k_end = min(U.k_begin + p.split_len, U.ctx);
+  U.t0 = U.k_begin / kTileK;
+  U.nt = (U.k_end - 1) / kTileK - U.t0 + 1;
 }
 
 }  // namespace
@@ -100,204 +156,280 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar0 = sbase + kOffBar;
+  const int pair = warp & (kPairs - 1);
+  const bool producer = warp < kPairs;
+  const uint32_t region = sbase + pair * kPairBytes;  // stages, then the two query tiles
+  const uint32_t qtile0 = region + kStages * kStageBytes;
+  UnitInfo* info = reinterpret_cast<UnitInfo*>(smem + kOffInfo + pair * 2 * kInfoBytes);
+  auto info_at = [&](int b) {
+    return reinterpret_cast<UnitInfo*>(reinterpret_cast<uint8_t*>(info) + b * kInfoBytes);
+  };
+  const uint32_t bar0 = sbase + kOffBar + pair * kBarsPerPair * 8;
   auto full = [&](int i) { return bar0 + 8 * i; };
   auto empty = [&](int i) { return bar0 + 8 * (kStages + i); };
-  const uint32_t merge_ready = bar0 + 8 * (2 * kStages);
-  const uint32_t merge_free = bar0 + 8 * (2 * kStages + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + 8 * (2 * kStages + 2));
+  auto q_full = [&](int b) { return bar0 + 8 * (2 * kStages + b); };
+  auto q_empty = [&](int b) { return bar0 + 8 * (2 * kStages + 2 + b); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kPairs * kBarsPerPair * 8);
   unsigned* status = p.status;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(full(i), 1);
-      mbar_init(empty(i), 4);
-    }
-    mbar_init(merge_ready, 128);
-    mbar_init(merge_free, 128);
-    *abort_flag = 0;
+  if (producer && lane == 0) {
+    for (int i = 0; i < kBarsPerPair; ++i) mbar_init(bar0 + 8 * i, 1);
+    if (pair == 0) *abort_flag = 0;
     fence_mbar_init();
   }
+  // split-KV with few enough sequences: enumerate only the units that have keys, full splits first
+  const bool ordered = p.max_splits > 1 && p.batch <= kMaxTable && p.cache_kind == MIMO_CACHE_PAGED;
+  int* tbl_full = reinterpret_cast<int*>(smem + kOffTbl);
+  int* tbl_part = tbl_full + kMaxTable + 1;
+  if (ordered && warp == kPairs) {
+    int carry_f = 0, carry_p = 0;
+    if (lane == 0) tbl_full[0] = tbl_part[0] = 0;
+    for (int base = 0; base < p.batch; base += 32) {
+      const int s = base + lane;
+      int keys = s < p.batch ? seq_keys(p, p.seq_lens[s]) : 0;
+      if (keys > p.max_splits * p.split_len) {  // a context beyond max_seq_len
+        atomicOr(status, MIMO_STATUS_BAD_INDEX);
+        keys = p.max_splits * p.split_len;
+      }
+      int f = keys / p.split_len, q = keys % p.split_len ? 1 : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int uf = __shfl_up_sync(0xffffffffu, f, d), uq = __shfl_up_sync(0xffffffffu, q, d);
+        if (lane >= d) {
+          f += uf;
+          q += uq;
+        }
+      }
+      if (s < p.batch) {
+        tbl_full[s + 1] = carry_f + f;
+        tbl_part[s + 1] = carry_p + q;
+      }
+      carry_f += __shfl_sync(0xffffffffu, f, 31);
+      carry_p += __shfl_sync(0xffffffffu, q, 31);
+    }
+  }
   __syncthreads();
-  const int n_units = p.batch * p.hkv * p.max_splits;
+  const int n_units = ordered ? (tbl_full[p.batch] + tbl_part[p.batch]) * p.hkv : p.batch * p.hkv * p.max_splits;
+  const int wp = blockIdx.x * kPairs + pair;
+  const int n_pairs = gridDim.x * kPairs;
+  auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
+  };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (producer) {
+    // ------------------------------------------------------------ producer warp
     if (lane == 0) {
+      tma_prefetch(&p.tm_q);
       tma_prefetch(&p.tm_k);
       tma_prefetch(&p.tm_v);
     }
-    int it = 0;
+    int it = 0, n = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      Unit U;
-      if (!unit_at(p, u, U)) continue;
-      // cache row of each tile of the unit (lane i: tile i); a unit spans at most 32 tiles
+    for (int u = wp; u < n_units && ok; u += n_pairs) {
+      UnitInfo U;
+      if (ordered) unit_ordered(p, tbl_full, tbl_part, u, U);
+      else if (!unit_at(p, u, U)) continue;
+      // cache row of page i of the unit in lane i (a unit spans at most 32 pages)
       int row_l = 0;
-      if (lane < U.nt) {
-        if (p.cache_kind == MIMO_CACHE_RING) {
-          row_l = U.s * kPage + kTile * lane;
-        } else {
-          const int pi = (U.t0 + lane) * kTile / kPage;
-          int page = pi < p.max_pages ? p.block_table[long(U.s) * p.max_pages + pi] : -1;
-          if (page < 0 || page >= p.num_pages) {
-            atomicOr(status, MIMO_STATUS_BAD_INDEX);
-            page = 0;
-          }
-          row_l = page * kPage + ((U.t0 + lane) * kTile) % kPage;
+      const int p0 = U.k_begin / kPage;
+      if (p.cache_kind == MIMO_CACHE_PAGED && lane <= (U.k_end - 1) / kPage - p0) {
+        const int pi = p0 + lane;
+        int page = pi < p.max_pages ? p.block_table[long(U.s) * p.max_pages + pi] : -1;
+        if (page < 0 || page >= p.num_pages) {
+          atomicOr(status, MIMO_STATUS_BAD_INDEX);
+          page = 0;
         }
+        row_l = page * kPage;
       }
+      // hand the unit to the consumer: fields, the rotary row at the query position, the query tile
+      const int b = n & 1;
+      if (n >= 2 && !(ok = wait_w(q_empty(b), ((n >> 1) - 1) & 1))) break;
+      UnitInfo* I = info_at(b);
+      float c, s;
+      rope_cos_sin(U.ctx - 1, p.rope.inv_freq[lane], &c, &s);
+      reinterpret_cast<float2*>(I + 1)[lane] = make_float2(c, s);
+      if (lane == 0) *I = U;
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t dst = qtile0 + b * kQBytes;
+        mbar_expect_tx(q_full(b), kQBytes);
+        const int h0 = U.g * p.group;
+        tma_load_3d(dst, &p.tm_q, q_full(b), 0, h0, U.s);
+        tma_load_3d(dst + kQChunk, &p.tm_q, q_full(b), 64, h0, U.s);
+        tma_load_3d(dst + 2 * kQChunk, &p.tm_q, q_full(b), 128, h0, U.s);
+      }
+      ++n;
       for (int t = 0; t < U.nt; ++t, ++it) {
-        const int row = __shfl_sync(0xffffffffu, row_l, t);
+        int row;
+        if (p.cache_kind == MIMO_CACHE_RING) {
+          row = U.s * kPage + kTileK * t;
+        } else {
+          const int key = (U.t0 + t) * kTileK;
+          row = __shfl_sync(0xffffffffu, row_l, key / kPage - p0) + key % kPage;
+        }
         const int st = it % kStages;
-        if (it >= kStages &&
-            !(ok = __all_sync(0xffffffffu, mbar_wait(empty(st), ((it / kStages) - 1) & 1, abort_flag, status,
-                                                     MIMO_STATUS_TIMEOUT))))
-          break;
+        if (it >= kStages && !(ok = wait_w(empty(st), ((it / kStages) - 1) & 1))) break;
         if (lane == 0) {
-          const uint32_t dst = sbase + st * kStageBytes;
+          const uint32_t dst = region + st * kStageBytes;
           mbar_expect_tx(full(st), kStageBytes);
           tma_load_3d(dst, &p.tm_k, full(st), 0, U.g, row);
-          tma_load_3d(dst + kKChunk, &p.tm_k, full(st), 64, U.g, row);
-          tma_load_3d(dst + 2 * kKChunk, &p.tm_k, full(st), 128, U.g, row);
-          tma_load_3d(dst + 3 * kKChunk, &p.tm_v, full(st), 0, U.g, row);
-          tma_load_3d(dst + 4 * kKChunk, &p.tm_v, full(st), 64, U.g, row);
+          tma_load_3d(dst + kChunk, &p.tm_k, full(st), 64, U.g, row);
+          tma_load_3d(dst + 2 * kChunk, &p.tm_k, full(st), 128, U.g, row);
+          tma_load_3d(dst + 3 * kChunk, &p.tm_v, full(st), 0, U.g, row);
+          tma_load_3d(dst + 4 * kChunk, &p.tm_v, full(st), 64, U.g, row);
         }
         __syncwarp();
       }
     }
+    if (ok) {
+      // end of the unit stream
+      const int b = n & 1;
+      if (n < 2 || (ok = wait_w(q_empty(b), ((n >> 1) - 1) & 1))) {
+        if (lane == 0) {
+          info_at(b)->nt = -1;
+          mbar_arrive(q_full(b));
+        }
+      }
+    }
     if (!ok && lane == 0) {
-      // let copies already in flight land before the CTA leaves
+      // let the copies already issued land before the CTA leaves
       int dummy = 0;
-      for (int i = 0; i < kStages; ++i) mbar_wait(full(i), 0, &dummy, nullptr, 0, 50000000ull);
+      for (int k = it - kStages < 0 ? 0 : it - kStages; k < it; ++k)
+        mbar_wait(full(k % kStages), (k / kStages) & 1, &dummy, nullptr, 0, 50000000ull);
+      for (int k = n - 2 < 0 ? 0 : n - 2; k < n; ++k)
+        mbar_wait(q_full(k & 1), (k >> 1) & 1, &dummy, nullptr, 0, 50000000ull);
     }
     return;
   }
 
-  // ------------------------------------------------------------ compute warps 1..4
-  const int cw = warp - 1;
-  const int tid = threadIdx.x - 32;  // 0..127
-  const int G = p.group;
+  // ------------------------------------------------------------ consumer warp
   const int q4 = lane & 3, r0 = lane >> 2, r1 = r0 + 8;
   const float c_log2 = p.scale_log2;
-  float* mw = reinterpret_cast<float*>(smem + kOffMerge);  // [4][16]
-  float* lw = mw + 4 * 16;                                 // [4][16]
-  float* ow = lw + 4 * 16;                                 // [4][16][128]
-  auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
-  };
-  int it = 0, n_done = 0;
-  bool ok = true;
-  for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-    Unit U;
-    if (!unit_at(p, u, U)) continue;
-    const int pos = U.ctx - 1;
-    // ---- query fragments (A of m16n8k16) for the G heads of KV head g, RoPE in registers
+  int it = 0;
+  for (int n = 0;; ++n) {
+    const int b = n & 1;
+    if (!wait_w(q_full(b), (n >> 1) & 1)) return;
+    const UnitInfo* I = info_at(b);
+    const int nt = I->nt;
+    if (nt < 0) return;
+    const int s = I->s, g = I->g, split = I->split, ctx = I->ctx, k_begin = I->k_begin, k_end = I->k_end,
+              t0 = I->t0;
+    // ---- query fragments (A of m16n8k16) from the swizzled tile; rows = heads of the group
     uint32_t qa[12][4];
     {
-      const uint16_t* q0 = p.q + (long(U.s) * kHq + U.g * G) * kDqk;
-      const bool v0 = r0 < G, v1 = r1 < G;
+      const uint32_t qt = qtile0 + b * kQBytes;
+      const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < 12; ++kk) {
-        const int c = 16 * kk + 2 * q4;
-        qa[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(q0 + r0 * kDqk + c) : 0u;
-        qa[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(q0 + r1 * kDqk + c) : 0u;
-        qa[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(q0 + r0 * kDqk + c + 8) : 0u;
-        qa[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(q0 + r1 * kDqk + c + 8) : 0u;
+        const int unit16 = ((kk & 3) * 2 + (lane >> 4)) ^ (row & 7);
+        ldsm_x4(qt + (kk >> 2) * kQChunk + row * 128 + unit16 * 16, qa[kk]);
       }
       // dims j < 32 (k-steps 0, 1) pair with dims j + 32 (k-steps 2, 3) in the same register slot
+      const float4* cs = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(I + 1));
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j0 = 16 * kk + 2 * q4 + ((e & 2) ? 8 : 0);
-          float c0, s0, c1, s1;
-          rope_cos_sin(pos, p.rope.inv_freq[j0], &c0, &s0);
-          rope_cos_sin(pos, p.rope.inv_freq[j0 + 1], &c1, &s1);
+          const float4 t = cs[j0 >> 1];  // (cos, sin) of frequencies j0, j0 + 1
           const uint32_t xw = qa[kk][e], yw = qa[kk + 2][e];
           const float x0 = lo_bf16(xw), x1 = hi_bf16(xw), y0 = lo_bf16(yw), y1 = hi_bf16(yw);
-          qa[kk][e] = pack2_f16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
-          qa[kk + 2][e] = pack2_f16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1);
+          qa[kk][e] = pack2_f16(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+          qa[kk + 2][e] = pack2_f16(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
         }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_empty(b));
+
     float m_r[2] = {-INFINITY, -INFINITY};
     float l_r[2] = {0.f, 0.f};
     float o[16][4];
 #pragma unroll
     for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-    for (int t = 0; t < U.nt; ++t, ++it) {
+    for (int t = 0; t < nt; ++t, ++it) {
       const int st = it % kStages;
-      if (!(ok = wait_w(full(st), (it / kStages) & 1))) break;
-      const uint32_t kb = sbase + st * kStageBytes;
-      const uint32_t vb = kb + 3 * kKChunk;
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (!wait_w(full(st), (it / kStages) & 1)) return;
+      const uint32_t kb = region + st * kStageBytes;
+      const uint32_t vb = kb + 3 * kChunk;
+      // two accumulators per key half (even / odd k-steps) halve the dependent MMA chain
+      float acc[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
       {
-        // B fragments of K^T: matrices (keys 0-7 | 8-15) x (dims lo 8 | hi 8) of this warp's 16 keys;
+        // B fragments of K^T: matrices (keys 0-7 | 8-15) x (dims lo 8 | hi 8);
         // rows are 128-byte swizzled (16-byte unit u of row k sits at u ^ (k & 7))
-        const int key = 16 * cw + (lane & 7) + (lane >> 4) * 8;
+        const int key = (lane & 7) + (lane >> 4) * 8;
         const int dhalf = (lane >> 3) & 1;
 #pragma unroll
         for (int kk = 0; kk < 12; ++kk) {
           const int unit16 = ((kk & 3) * 2 + dhalf) ^ (key & 7);
-          uint32_t b[4];
-          ldsm_x4(kb + (kk >> 2) * kKChunk + key * 128 + unit16 * 16, b);
+          uint32_t bf[4];
+          ldsm_x4(kb + (kk >> 2) * kChunk + key * 128 + unit16 * 16, bf);
+          float* a0 = acc[kk & 1];
+          float* a1 = acc[2 + (kk & 1)];
           if (kk < 4) {
-            mma_f16(acc0, qa[kk], b[0], b[1]);
-            mma_f16(acc1, qa[kk], b[2], b[3]);
+            mma_f16(a0, qa[kk], bf[0], bf[1]);
+            mma_f16(a1, qa[kk], bf[2], bf[3]);
           } else {
-            mma_bf16(acc0, qa[kk], b[0], b[1]);
-            mma_bf16(acc1, qa[kk], b[2], b[3]);
+            mma_bf16(a0, qa[kk], bf[0], bf[1]);
+            mma_bf16(a1, qa[kk], bf[2], bf[3]);
           }
         }
+      }
+      float s0[4], s1[4];  // keys 2q4, 2q4+1 (rows r0, r0, r1, r1) and the same + 8
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        s0[i] = acc[0][i] + acc[1][i];
+        s1[i] = acc[2][i] + acc[3][i];
       }
       // positions of this thread's four key columns and their visibility
       bool vis[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int col = 16 * cw + ((e & 2) ? 8 : 0) + 2 * q4 + (e & 1);  // within the 64-key tile
+        const int col = ((e & 2) ? 8 : 0) + 2 * q4 + (e & 1);  // within the 16-key tile
         int kp;
         if (p.cache_kind == MIMO_CACHE_RING) {
-          const int slot = kTile * t + col;
-          const int base = U.ctx - kPage;  // the ring holds positions base .. ctx-1
+          const int slot = kTileK * t + col;
+          const int base = ctx - kPage;  // the ring holds positions base .. ctx-1
           kp = base + (((slot - base) % kPage) + kPage) % kPage;
         } else {
-          kp = (U.t0 + t) * kTile + col;
+          kp = (t0 + t) * kTileK + col;
         }
-        vis[e] = kp >= U.k_begin && kp < U.k_end;
+        vis[e] = kp >= k_begin && kp < k_end;
       }
-      if (!vis[0]) acc0[0] = acc0[2] = -INFINITY;
-      if (!vis[1]) acc0[1] = acc0[3] = -INFINITY;
-      if (!vis[2]) acc1[0] = acc1[2] = -INFINITY;
-      if (!vis[3]) acc1[1] = acc1[3] = -INFINITY;
-      float mx0 = fmaxf(fmaxf(acc0[0], acc0[1]), fmaxf(acc1[0], acc1[1]));
-      float mx1 = fmaxf(fmaxf(acc0[2], acc0[3]), fmaxf(acc1[2], acc1[3]));
+      if (!vis[0]) s0[0] = s0[2] = -INFINITY;
+      if (!vis[1]) s0[1] = s0[3] = -INFINITY;
+      if (!vis[2]) s1[0] = s1[2] = -INFINITY;
+      if (!vis[3]) s1[1] = s1[3] = -INFINITY;
+      float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
+      float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
       const float mn0 = fmaxf(m_r[0], mx0 * c_log2), mn1 = fmaxf(m_r[1], mx1 * c_log2);
-      // all keys of this warp's share of a tile may be masked (tile edges): reference 0 then
+      // a tile may be fully masked (split edges): reference 0 then
       const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float a0 = ex2(m_r[0] - mu0), a1 = ex2(m_r[1] - mu1);
+      const float al0 = ex2(m_r[0] - mu0), al1 = ex2(m_r[1] - mu1);
       m_r[0] = mn0;
       m_r[1] = mn1;
       float p0[4], p1[4];
-      p0[0] = ex2(fmaf(acc0[0], c_log2, -mu0));
-      p0[1] = ex2(fmaf(acc0[1], c_log2, -mu0));
-      p0[2] = ex2(fmaf(acc0[2], c_log2, -mu1));
-      p0[3] = ex2(fmaf(acc0[3], c_log2, -mu1));
-      p1[0] = ex2(fmaf(acc1[0], c_log2, -mu0));
-      p1[1] = ex2(fmaf(acc1[1], c_log2, -mu0));
-      p1[2] = ex2(fmaf(acc1[2], c_log2, -mu1));
-      p1[3] = ex2(fmaf(acc1[3], c_log2, -mu1));
-      l_r[0] = l_r[0] * a0 + p0[0] + p0[1] + p1[0] + p1[1];
-      l_r[1] = l_r[1] * a1 + p0[2] + p0[3] + p1[2] + p1[3];
+      p0[0] = ex2(fmaf(s0[0], c_log2, -mu0));
+      p0[1] = ex2(fmaf(s0[1], c_log2, -mu0));
+      p0[2] = ex2(fmaf(s0[2], c_log2, -mu1));
+      p0[3] = ex2(fmaf(s0[3], c_log2, -mu1));
+      p1[0] = ex2(fmaf(s1[0], c_log2, -mu0));
+      p1[1] = ex2(fmaf(s1[1], c_log2, -mu0));
+      p1[2] = ex2(fmaf(s1[2], c_log2, -mu1));
+      p1[3] = ex2(fmaf(s1[3], c_log2, -mu1));
+      l_r[0] = l_r[0] * al0 + p0[0] + p0[1] + p1[0] + p1[1];
+      l_r[1] = l_r[1] * al1 + p0[2] + p0[3] + p1[2] + p1[3];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        o[i][0] *= a0;
-        o[i][1] *= a0;
-        o[i][2] *= a1;
-        o[i][3] *= a1;
+        o[i][0] *= al0;
+        o[i][1] *= al0;
+        o[i][2] *= al1;
+        o[i][3] *= al1;
       }
       uint32_t pa[4];
       pa[0] = pack2_bf16(p0[0], p0[1]);
@@ -306,96 +438,58 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       pa[3] = pack2_bf16(p1[2], p1[3]);
       {
         // B fragments of V (trans): matrices (keys 0-7 | 8-15) x (dims d0 .. d0+7 | d0+8 ..)
-        const int key = 16 * cw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
         const int dq = lane >> 4;
 #pragma unroll
         for (int n2 = 0; n2 < 8; ++n2) {
           const int unit16 = ((n2 & 3) * 2 + dq) ^ (key & 7);
-          uint32_t b[4];
-          ldsm_x4_t(vb + (n2 >> 2) * kKChunk + key * 128 + unit16 * 16, b);
-          mma_bf16(o[2 * n2], pa, b[0], b[1]);
-          mma_bf16(o[2 * n2 + 1], pa, b[2], b[3]);
+          uint32_t bf[4];
+          ldsm_x4_t(vb + (n2 >> 2) * kChunk + key * 128 + unit16 * 16, bf);
+          mma_bf16(o[2 * n2], pa, bf[0], bf[1]);
+          mma_bf16(o[2 * n2 + 1], pa, bf[2], bf[3]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(st));
     }
-    if (!ok) break;
 
-    // ---- merge the 4 warps (rows = heads) and write the unit's result
+    // ---- the unit's result: rows r0, r1 are heads g*G + r0 / r1 (valid below G)
     l_r[0] += __shfl_xor_sync(0xffffffffu, l_r[0], 1);
     l_r[0] += __shfl_xor_sync(0xffffffffu, l_r[0], 2);
     l_r[1] += __shfl_xor_sync(0xffffffffu, l_r[1], 1);
     l_r[1] += __shfl_xor_sync(0xffffffffu, l_r[1], 2);
-    if (n_done > 0 && !(ok = wait_w(merge_free, (n_done - 1) & 1))) break;
-    if (q4 == 0) {
-      mw[cw * 16 + r0] = m_r[0];
-      mw[cw * 16 + r1] = m_r[1];
-      lw[cw * 16 + r0] = l_r[0];
-      lw[cw * 16 + r1] = l_r[1];
-    }
+    const int G = p.group;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int d = nt * 8 + 2 * q4;
-      *reinterpret_cast<float2*>(ow + (cw * 16 + r0) * kDv + d) = make_float2(o[nt][0], o[nt][1]);
-      *reinterpret_cast<float2*>(ow + (cw * 16 + r1) * kDv + d) = make_float2(o[nt][2], o[nt][3]);
-    }
-    mbar_arrive(merge_ready);
-    if (!(ok = wait_w(merge_ready, n_done & 1))) break;
-    {
-      const int row = tid >> 3, d0 = (tid & 7) * 16;
-      if (row < G) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[w * 16 + row]);
-        const float Mu = M == -INFINITY ? 0.f : M;
-        float wgt[4], L = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          wgt[w] = ex2(mw[w * 16 + row] - Mu);
-          L += wgt[w] * lw[w * 16 + row];
+    for (int half = 0; half < 2; ++half) {
+      const int row = half ? r1 : r0;
+      if (row >= G) continue;
+      const int h = g * G + row;
+      const float M = m_r[half], L = l_r[half];
+      if (p.max_splits == 1) {
+        float M2 = M, L2 = L, f = 1.f;
+        if (p.sink) {
+          const float sl = p.sink[h] * kLog2e;
+          M2 = fmaxf(M, sl);
+          f = ex2(M - M2);
+          L2 = L * f + ex2(sl - M2);
         }
-        float acc[16];
+        const float sc = p.v_scale * f / L2;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (long(s) * kHq + h) * kDv + 2 * q4);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float v = 0.f;
+        for (int i = 0; i < 16; ++i) dst[i * 4] = pack2_bf16(o[i][2 * half] * sc, o[i][2 * half + 1] * sc);
+        if (p.lse && q4 == 0) p.lse[long(s) * kHq + h] = (M2 + __log2f(L2)) * kLn2;
+      } else {
+        float* dst = p.ws_o + ((long(s) * kHq + h) * p.max_splits + split) * kDv + 2 * q4;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) v += wgt[w] * ow[(w * 16 + row) * kDv + d0 + i];
-          acc[i] = v;
-        }
-        const int h = U.g * G + row;
-        if (p.max_splits == 1) {
-          float M2 = Mu, L2 = L, f = 1.f;
-          if (p.sink) {
-            const float sl = p.sink[h] * kLog2e;
-            M2 = fmaxf(Mu, sl);
-            f = ex2(Mu - M2);
-            L2 = L * f + ex2(sl - M2);
-          }
-          const float sc = p.v_scale * f / L2;
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (long(U.s) * kHq + h) * kDv + d0);
-#pragma unroll
-          for (int i = 0; i < 2; ++i)
-            dst[i] = make_uint4(pack2_bf16(acc[8 * i] * sc, acc[8 * i + 1] * sc),
-                                pack2_bf16(acc[8 * i + 2] * sc, acc[8 * i + 3] * sc),
-                                pack2_bf16(acc[8 * i + 4] * sc, acc[8 * i + 5] * sc),
-                                pack2_bf16(acc[8 * i + 6] * sc, acc[8 * i + 7] * sc));
-          if (p.lse && d0 == 0) p.lse[long(U.s) * kHq + h] = (M2 + __log2f(L2)) * kLn2;
-        } else {
-          float* dst = p.ws_o + ((long(U.s) * kHq + h) * p.max_splits + U.split) * kDv + d0;
-#pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
-          if (d0 == 0) {
-            float* ml = p.ws_ml + ((long(U.s) * kHq + h) * p.max_splits + U.split) * 2;
-            ml[0] = M;
-            ml[1] = L;
-          }
+        for (int i = 0; i < 16; ++i)
+          *reinterpret_cast<float2*>(dst + i * 8) = make_float2(o[i][2 * half], o[i][2 * half + 1]);
+        if (q4 == 0) {
+          float* ml = p.ws_ml + ((long(s) * kHq + h) * p.max_splits + split) * 2;
+          ml[0] = M;
+          ml[1] = L;
         }
       }
     }
-    mbar_arrive(merge_free);
-    ++n_done;
   }
 }
 
@@ -411,7 +505,11 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const __grid_consta
     return;
   }
   const int lo = p.window > 0 ? max(0, ctx - p.window) : 0;
-  const int nsplit = (ctx - lo + p.split_len - 1) / p.split_len;
+  int nsplit = (ctx - lo + p.split_len - 1) / p.split_len;
+  if (nsplit > p.max_splits) {  // a context beyond max_seq_len: its extra keys were not attended
+    if (lane == 0 && h == 0) atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
+    nsplit = p.max_splits;
+  }
   const float* ml = p.ws_ml + (long(s) * kHq + h) * p.max_splits * 2;
   float M = -INFINITY;
   for (int i = lane; i < nsplit; i += 32) M = fmaxf(M, ml[2 * i]);
@@ -443,14 +541,18 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const __grid_consta
   if (p.lse && lane == 0) p.lse[long(s) * kHq + h] = (M + __log2f(L)) * kLn2;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* ev_begin, void* ev_end) {
   cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const long units = long(p.batch) * p.hkv * p.max_splits;
-  const int grid = int(units < sms ? units : sms);
+  const long ctas = (units + kPairs - 1) / kPairs;
+  const int grid = int(ctas < sms ? ctas : sms);
+  if (ev_begin && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s)) != cudaSuccess) return e;
   decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
   e = cudaGetLastError();
-  if (e != cudaSuccess || p.max_splits <= 1) return e;
+  if (e != cudaSuccess) return e;
+  if (ev_end && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s)) != cudaSuccess) return e;
+  if (p.max_splits <= 1) return e;
   const long warps = long(p.batch) * kHq;
   decode_combine_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, s>>>(p);
   return cudaGetLastError();

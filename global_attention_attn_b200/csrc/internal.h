@@ -36,8 +36,9 @@ struct AppendParams {
 };
 
 struct DecodeParams {
-  CUtensorMap tm_k;  // key cache rows [rows, Hkv, 192], box {64, 1, 64}
-  CUtensorMap tm_v;  // value cache rows [rows, Hkv, 128], box {64, 1, 64}
+  CUtensorMap tm_q;  // queries [batch, 64, 192], box {64, 16, 1}
+  CUtensorMap tm_k;  // key cache rows [rows, Hkv, 192], box {64, 1, 16}
+  CUtensorMap tm_v;  // value cache rows [rows, Hkv, 128], box {64, 1, 16}
   int batch, hkv, group;  // group = 64 / hkv
   int window;
   int split_len, max_splits;
@@ -109,7 +110,8 @@ struct RopeKParams {
 };
 
 cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s);
-cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s);
+// ev_begin / ev_end: optional cudaEvent_t recorded around the decode kernel (not the combine)
+cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* ev_begin, void* ev_end);
 cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s);
 // kind 0: sliding window (G=8 heads x 16 rows, one 144-key tile); kind 1: global (G=16 x 8 rows, 128-key tiles)
 cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s);

@@ -893,66 +893,116 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
       const float sink = sink_l2[head];
       float m_use, la[4];
       if (band) {
-        // Columns 16..127 are visible to every row.  S is read in chunks of 32 columns
-        // (the last one 16): the edge columns are the first half of chunk 0 and all of
-        // chunk 4, chunks 1..3 need no mask.  Each chunk's TMEM load is issued before
-        // the previous chunk is processed (two register buffers).
+        // Columns 16..127 are visible to every row; the edge columns are the first half of
+        // chunk 0 and all of chunk 4 (chunks of 32 columns, the last one 16).  One pass over
+        // S: chunk 4 (keys q0 .. q0+15) holds every row's own key, so its visible maximum
+        // (with the sink) is the reference m_use of the exponentials of all chunks; the
+        // softmax needs no exact row maximum, only no overflow, and the LSE is
+        // m_use + log2(sum).  A chunk whose sum overflows 2^64 (a logit far above the
+        // reference) raises m_use to its maximum and rescales the P already written.
+        // TMEM loads run one chunk ahead (two register buffers).
         uint32_t buf[2][32];
-        float mxa[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         auto ld = [&](int h, uint32_t* d) {
           if (h < 4) tmem_ld32(t_lane + 32 * h, d);
           else tmem_ld16(t_lane + 128, d);
         };
         auto edge_col = [&](int h, int c) { return (h == 0 && c < 16) || h == 4; };
-        auto max_chunk = [&](const uint32_t* sr, int h) {
-#pragma unroll
-          for (int c = 0; c < (h < 4 ? 32 : 16); ++c) {
-            const int cc = 32 * h + c;
-            if (!edge_col(h, c) || (cc >= ca && cc <= ce)) mxa[c & 3] = fmaxf(mxa[c & 3], __uint_as_float(sr[c]));
-          }
+        auto vis_col = [&](int h, int c) {
+          const int cc = 32 * h + c;
+          return !edge_col(h, c) || (cc >= ca && cc <= ce);
         };
-        ld(0, buf[0]);
-        tmem_wait_ld_r32(buf[0]);
+        auto chunk_max = [&](const uint32_t* sr, int h) {
+          float mx = -INFINITY;
 #pragma unroll
-        for (int h = 0; h < 5; ++h) {
-          if (h < 4) ld(h + 1, buf[(h + 1) & 1]);
-          else ld(0, buf[1]);  // chunk 0 again, for the exponentials
-          max_chunk(buf[h & 1], h);
-          if (h == 3) tmem_wait_ld_r16_after(buf[0], mxa[0], mxa[1], mxa[2], mxa[3]);
-          else tmem_wait_ld_r32_after(buf[(h + 1) & 1], mxa[0], mxa[1], mxa[2], mxa[3]);
+          for (int c = 0; c < (h < 4 ? 32 : 16); ++c)
+            if (vis_col(h, c)) mx = fmaxf(mx, __uint_as_float(sr[c]));
+          return mx;
+        };
+        ld(4, buf[0]);
+        ld(0, buf[1]);
+        tmem_wait_ld_r16(buf[0]);
+        {
+          const float m_row = fmaxf(sink, chunk_max(buf[0], 4) * c_log2);
+          m_use = m_row == -INFINITY ? 0.f : m_row;
         }
-        const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
-        const float m_row = fmaxf(sink, mx * c_log2);
-        m_use = m_row == -INFINITY ? 0.f : m_row;
+        const uint64_t cl2 = pack_f32x2(c_log2, c_log2);
         uint64_t la2 = pack_f32x2(p.sink ? ex2(sink - m_use) : 0.f, 0.f);
-        const uint64_t cl2 = pack_f32x2(c_log2, c_log2), nm2 = pack_f32x2(-m_use, -m_use);
-        auto exp_chunk = [&](const uint32_t* sr, int h) {
+        // exponentials of one chunk into packed bf16 words; returns the chunk's sum
+        auto exp_chunk = [&](const uint32_t* sr, int h, uint32_t* pk) {
+          const uint64_t nm2 = pack_f32x2(-m_use, -m_use);
+          uint64_t sum2 = pack_f32x2(0.f, 0.f);
 #pragma unroll
-          for (int g = 0; g < (h < 4 ? 32 : 16); g += 16) {  // 16 columns -> 8 packed words -> one TMEM store
-            uint32_t pk[8];
-#pragma unroll
-            for (int c = g; c < g + 16; c += 2) {
-              const uint64_t t = fma_f32x2(pack_f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, nm2);
-              float p0 = ex2(lo_f32(t)), p1 = ex2(hi_f32(t));
-              if (edge_col(h, c)) {
-                const int cc = 32 * h + c;
-                p0 = (cc >= ca && cc <= ce) ? p0 : 0.f;
-                p1 = (cc + 1 >= ca && cc + 1 <= ce) ? p1 : 0.f;
-              }
-              la2 = add_f32x2(la2, pack_f32x2(p0, p1));
-              pk[(c - g) / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < (h < 4 ? 32 : 16); c += 2) {
+            const uint64_t t = fma_f32x2(pack_f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, nm2);
+            float p0 = ex2(lo_f32(t)), p1 = ex2(hi_f32(t));
+            if (edge_col(h, c)) {
+              p0 = vis_col(h, c) ? p0 : 0.f;
+              p1 = vis_col(h, c + 1) ? p1 : 0.f;
             }
-            tmem_st8(t_lane + (32 * h + g) / 2, pk);
+            sum2 = add_f32x2(sum2, pack_f32x2(p0, p1));
+            pk[c / 2] = pack_bf16x2(p0, p1);
           }
+          return lo_f32(sum2) + hi_f32(sum2);
         };
-        // chunk 0 is in buf[1]
+        // rare: rows whose chunk sum overflowed take the chunk's maximum as the new
+        // reference; P columns [0, written) in TMEM, the held chunk-4 words and the running
+        // sum are scaled down to it (warp-uniform loop: TMEM access is warp-collective)
+        uint32_t pk4[8];
+        auto raise_ref = [&](bool over, const uint32_t* sr, int h, int written) {
+          tmem_wait_st();
+          float f = 1.f;
+          if (over) {
+            const float m_new = fmaxf(m_use, chunk_max(sr, h) * c_log2);
+            f = ex2(m_use - m_new);
+            m_use = m_new;
+          }
+          const uint64_t f2 = pack_f32x2(f, f);
+          la2 = mul_f32x2(la2, f2);
 #pragma unroll
-        for (int h = 0; h < 5; ++h) {
-          if (h < 4) ld(h + 1, buf[h & 1]);
-          exp_chunk(buf[(h + 1) & 1], h);
-          if (h == 3) tmem_wait_ld_r16_after(buf[h & 1], la2);
-          else if (h < 3) tmem_wait_ld_r32_after(buf[h & 1], la2);
+          for (int i = 0; i < 8; ++i) {
+            const uint64_t t = mul_f32x2(pack_f32x2(lo_bf16(pk4[i]), hi_bf16(pk4[i])), f2);
+            pk4[i] = pack_bf16x2(lo_f32(t), hi_f32(t));
+          }
+#pragma unroll 1
+          for (int c0 = 0; c0 < written; c0 += 8) {
+            uint32_t w[8];
+            tmem_ld8(t_lane + c0, w);
+            tmem_wait_ld_r8(w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint64_t t = mul_f32x2(pack_f32x2(lo_bf16(w[i]), hi_bf16(w[i])), f2);
+              w[i] = pack_bf16x2(lo_f32(t), hi_f32(t));
+            }
+            tmem_st8(t_lane + c0, w);
+          }
+          tmem_wait_st();
+        };
+        constexpr float kOver = 18446744073709551616.f;  // 2^64
+        {
+          float sum = exp_chunk(buf[0], 4, pk4);
+          if (__any_sync(0xffffffffu, !(sum <= kOver))) {
+            raise_ref(!(sum <= kOver), buf[0], 4, 0);
+            sum = exp_chunk(buf[0], 4, pk4);
+          }
+          la2 = add_f32x2(la2, pack_f32x2(sum, 0.f));
         }
+        tmem_wait_ld_r32(buf[1]);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint32_t* sr = buf[(h + 1) & 1];
+          if (h < 3) ld(h + 1, buf[h & 1]);
+          uint32_t pk[16];
+          float sum = exp_chunk(sr, h, pk);
+          if (__any_sync(0xffffffffu, !(sum <= kOver))) {
+            raise_ref(!(sum <= kOver), sr, h, 16 * h);
+            sum = exp_chunk(sr, h, pk);
+          }
+          tmem_st8(t_lane + 16 * h, pk);
+          tmem_st8(t_lane + 16 * h + 8, pk + 8);
+          if (h < 3) tmem_wait_ld_r32_after(buf[h & 1], la2);
+          la2 = add_f32x2(la2, pack_f32x2(sum, 0.f));
+        }
+        tmem_st8(t_lane + 64, pk4);
         la[0] = lo_f32(la2);
         la[1] = hi_f32(la2);
         la[2] = la[3] = 0.f;

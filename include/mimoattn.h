@@ -126,6 +126,12 @@ typedef struct {
   float* lse;
   void* workspace;
   size_t workspace_bytes;
+  /* Optional timing hooks: cudaEvent_t handles or NULL.  When set, they are
+   * recorded on `stream` immediately before the first and after the last
+   * launch of the attention kernel itself (not the key pre-pass), so that
+   * cudaEventElapsedTime gives that kernel's device time. */
+  void* ev_kernel_begin;
+  void* ev_kernel_end;
 } mimo_prefill_args;
 
 /* Bytes of workspace mimo_attn_prefill needs for these sizes. */
@@ -160,6 +166,12 @@ typedef struct {
   float* lse;
   void* workspace;
   size_t workspace_bytes;
+  /* Optional timing hooks: cudaEvent_t handles or NULL.  When set, they are
+   * recorded on `stream` immediately before the first and after the last
+   * launch of the attention kernel itself (not the split combine pass), so that
+   * cudaEventElapsedTime gives that kernel's device time. */
+  void* ev_kernel_begin;
+  void* ev_kernel_end;
 } mimo_decode_args;
 
 /* Bytes of workspace mimo_attn_decode needs (split-KV partials). */

@@ -117,6 +117,41 @@ def test_decode_split_boundaries():
     assert M.status_poll() == 0
 
 
+def _shared_page_decode(seed, B, ctx_range, pool, layer):
+    """Decode over a small page pool that the block tables share (prefix-shared pages):
+    large batches without a large cache."""
+    ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
+    maxp = int((ctx.max() + 127) // 128)
+    bt = synth.randint(synth.stream_seed(seed, 1), B * maxp, 0, pool - 1).astype(np.int32).reshape(B, maxp)
+    h = layer.num_kv_heads
+    return configs.Decode(layer, configs.bf16_normal(seed, 2, (B, 64, 192)), ctx,
+                          configs.cached_keys(seed, 3, (pool, 128, h, 192)),
+                          configs.bf16_normal(seed, 4, (pool, 128, h, 128)), block_table=bt)
+
+
+def test_decode_large_batch_shared_pages():
+    """More than 1024 sequences with several splits each: the split units are enumerated
+    densely instead of from the per-sequence table."""
+    import torch
+    cfg = _shared_page_decode(601, 1100, (513, 1600), 24, configs.global_layer())
+    out, lse = decode_cfg(cfg)
+    seqs = np.array(sorted(set([0, 1023, 1024, 1099] + list(synth.permutation(602, 1100)[:8]))), np.int32)
+    ro, rl = oracle.decode(cfg, seqs=seqs)
+    idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "decode 1100 sequences, shared pages")
+
+
+def test_decode_paged_window_unaligned_splits():
+    """A window on the paged cache: splits start mid-page and mid-tile."""
+    sink = synth.normal_f32(synth.stream_seed(603, 9), (64,))
+    for window in (1000, 300):
+        layer = configs.Layer("swa", 4, 1e7, window, sink)
+        cfg = _shared_page_decode(604 + window, 12, (200, 3000), 40, layer)
+        out, lse = decode_cfg(cfg)
+        ro, rl = oracle.decode(cfg)
+        parity(out, lse, ro, rl, f"paged decode, window {window}")
+
+
 @pytest.fixture(scope="module")
 def cfg3():
     return configs.config3()
