@@ -39,9 +39,10 @@ FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) p
 # The step's dominant kernel (about 97% of the step's device time in the ncu launch list).
 DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
-# workload, from the ncu capture summarised in profiles/; absent until the current kernel has
-# been captured.
-TRAFFIC_BYTES = {}
+# workload, from the ncu capture summarised in profiles/prefill_swa_kernel_2x4096_full.md
+# (kernel at commit 8eb4a8c): 249.65 MB read + 97.91 MB written for 2 x 4096 tokens, scaled
+# by tokens to the 40696-token workload.  Removed whenever the kernel changes.
+TRAFFIC_BYTES = {"prefill_swa_kernel": int((249.653504e6 + 97.910016e6) * 40696 / 8192)}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
@@ -80,17 +81,24 @@ def decode_counts(cfg):
 
 
 def chunked_counts(cfg):
+    """Algorithmic FLOP and bytes of a chunked prefill (workloads.configs.Chunked), any number
+    of sequences: queries and outputs once, every key the chunk attends once per KV head, and
+    for a paged layer the append (the chunk's keys and values read and written)."""
     L = cfg.layer
-    n = int(cfg.cu_new[-1])
-    start = int(cfg.start[0])
-    pos = start + np.arange(n, dtype=np.int64)
-    vis = np.minimum(pos + 1, L.window) if L.window else pos + 1
-    ctx = start + n
-    keys_read = (min(ctx, n + L.window - 1) if L.window else ctx)
+    lens = np.diff(cfg.cu_new).astype(np.int64)
+    pairs = keys_read = 0
+    for s in range(len(lens)):
+        start, n = int(cfg.start[s]), int(lens[s])
+        pos = start + np.arange(n, dtype=np.int64)
+        vis = np.minimum(pos + 1, L.window) if L.window else pos + 1
+        pairs += int(vis.sum())
+        ctx = start + n
+        keys_read += min(ctx, n + L.window - 1) if L.window else ctx
+    n = int(lens.sum())
     by = n * 64 * (192 * 2 + 128 * 2 + 4) + keys_read * L.num_kv_heads * (192 + 128) * 2
     if cfg.paged:
-        by += n * L.num_kv_heads * (192 + 128) * 2 * 2  # the append reads the chunk and writes it
-    return int(vis.sum()) * 64 * FLOP_PER_PAIR, by
+        by += n * L.num_kv_heads * (192 + 128) * 2 * 2
+    return pairs * 64 * FLOP_PER_PAIR, by
 
 
 def roofline_us(flops, by, hbm, tf):
@@ -282,22 +290,24 @@ class Chunked:
         self.sink = dev_f32(L.sink)
         self.out = torch.empty((n, 64, 128), dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty((n, 64), dtype=torch.float32, device="cuda")
+        lens = np.diff(cfg.cu_new)
+        B = len(lens)
         if cfg.paged:
             self.bt = dev_i32(cfg.block_table)
-            self.pos = dev_i32(cfg.start[0] + np.arange(n))
-            self.seq = dev_i32(np.zeros(n))
-            self.ctx = dev_i32(cfg.start + n)
+            self.pos = dev_i32(np.concatenate([cfg.start[s] + np.arange(lens[s]) for s in range(B)]))
+            self.seq = dev_i32(np.repeat(np.arange(B), lens))
+            self.ctx = dev_i32(cfg.start + lens)
             self.ws = None
         else:
             self.start = dev_i32(cfg.start)
-            w = M.prefill_workspace_size(1, n, n, L.num_kv_heads, M.MIMO_CACHE_RING)
+            w = M.prefill_workspace_size(B, n, n, L.num_kv_heads, M.MIMO_CACHE_RING)
             self.ws = torch.empty(w, dtype=torch.uint8, device="cuda")
 
     def __call__(self):
         M, L, cfg = self.M, self.cfg.layer, self.cfg
         if cfg.paged:
             M.mimo_kv_append(self.k, self.v, self.pos, self.seq, rope_base=L.rope_base, cache_kind=M.MIMO_CACHE_PAGED,
-                             k_cache=self.kc, v_cache=self.vc, num_seqs=1, block_table=self.bt,
+                             k_cache=self.kc, v_cache=self.vc, num_seqs=len(cfg.start), block_table=self.bt,
                              num_pages=cfg.k_cache.shape[0])
             M.mimo_attn_prefill(self.q, None, None, self.cu, None, num_kv_heads=L.num_kv_heads, rope_base=L.rope_base,
                                 window=L.window, sink=self.sink, cache_lens=self.ctx, cache_kind=M.MIMO_CACHE_PAGED,
@@ -526,7 +536,17 @@ def main():
             e["GB/s"] = bd / (td * 1e-3) / 1e9
             per[name] = e
             del w
-        del sw, gl
+        # speculative verification: 4 draft tokens per sequence on the config-3 caches
+        vg, vs = configs.verify(B=64, q_len=4, decode=gl)
+        for name, c in (("global_verify_b64_q4", vg), ("swa_verify_b64_q4", vs)):
+            fc, bc = chunked_counts(c)
+            w = Chunked(c)
+            for _ in range(3):
+                w()
+            tc = event_time_ms(w, 10, flush=flush) / 10
+            per[name] = _entry(fc, bc, tc, hbm, tf_burst, "L2 flushed before each call")
+            del w
+        del sw, gl, vg, vs
         torch.cuda.empty_cache()
         g4, s4 = configs.config4()
         for name, c in (("global_chunk_8192_on_120832", g4), ("swa_chunk_8192_on_120832", s4)):

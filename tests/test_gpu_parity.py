@@ -265,6 +265,35 @@ def test_chunked_config4():
 
 # ----------------------------------------------------------------------------- cross-path
 
+# ----------------------------------------------------------------------------- speculative verification
+
+@pytest.mark.parametrize("q_len", [2, 5, 8])
+def test_verify_draft_tokens(q_len):
+    """q_len draft tokens per sequence scored against the cache: the global layer appends them
+    to the paged cache and runs the chunked prefill over it; the sliding layer reads the prefix
+    tail from the ring and the drafts from the new rows."""
+    glb, swa = configs.verify(seed=700 + q_len, B=12, q_len=q_len, ctx_range=(q_len + 1, 3000))
+    for cfg in (glb, swa):
+        out, lse = chunked_cfg(cfg)
+        ro, rl = oracle.chunked(cfg, rows=np.arange(int(cfg.cu_new[-1])))
+        parity(out, lse, ro, rl, cfg.name)
+
+
+def test_verify_config3_scale(cfg3):
+    """Verification at the decode workload's scale (64 sequences, contexts up to 64K) on the
+    config-3 caches, checked on the rows of 4 sampled sequences."""
+    import torch
+    _, gl = cfg3
+    glb, swa = configs.verify(B=64, q_len=4, decode=gl)
+    seqs = np.array([0, 17, 42, 63])
+    rows = (seqs[:, None] * 4 + np.arange(4)[None, :]).reshape(-1)
+    for cfg in (glb, swa):
+        out, lse = chunked_cfg(cfg)
+        ro, rl = oracle.chunked(cfg, rows=rows)
+        idx = torch.as_tensor(rows, dtype=torch.long, device=out.device)
+        parity(out[idx], lse[idx], ro, rl, cfg.name)
+
+
 def test_decode_matches_last_prefill_row():
     """Appending a sequence to the caches and decoding its last token gives the last prefill row."""
     import torch

@@ -237,6 +237,38 @@ def config3(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536)) -> 
     return swa, glb
 
 
+def verify(seed: int = BASE_SEED + 5, B: int = 64, q_len: int = 4, ctx_range=(4096, 65536),
+           decode: Decode | None = None) -> tuple[Chunked, Chunked]:
+    """Speculative-decoding verification: each sequence scores q_len draft tokens at
+    positions [ctx - q_len, ctx) after a cached prefix of ctx - q_len tokens, for the
+    global layer (paged cache, the drafts appended first) and the SWA layer (ring holding
+    the 128 prefix positions before the drafts).  With `decode` (a global-layer Decode of
+    config 3) its contexts, block tables and cache are reused; the drafts then overwrite
+    the cache rows of the last q_len positions when they are appended."""
+    if decode is None:
+        ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
+        bt, pool = paged_layout(seed, 10, ctx)
+        kc = cached_keys(seed, 12, (pool, PAGE, 4, DQK))
+        vc = bf16_normal(seed, 13, (pool, PAGE, 4, DV))
+    else:
+        ctx, bt, kc, vc = decode.ctx, decode.block_table, decode.k_cache, decode.v_cache
+    B = len(ctx)
+    assert int(ctx.min()) >= q_len
+    start = (ctx - q_len).astype(np.int32)
+    cu = (np.arange(B + 1) * q_len).astype(np.int32)
+    n = B * q_len
+    glb = Chunked(global_layer(), bf16_normal(seed, 1, (n, HQ, DQK)), bf16_normal(seed, 2, (n, 4, DQK)),
+                  bf16_normal(seed, 3, (n, 4, DV)), cu, start, kc, vc, block_table=bt,
+                  name=f"global_verify_b{B}_q{q_len}")
+    # every ring slot holds a prefix position (slot p % 128 for p in [start - 128, start));
+    # slots of positions below 0 are never visible
+    Ls = swa_layer(synth.normal_f32(synth.stream_seed(seed, 24), (HQ,)))
+    swa = Chunked(Ls, bf16_normal(seed, 21, (n, HQ, DQK)), bf16_normal(seed, 22, (n, 8, DQK)),
+                  bf16_normal(seed, 23, (n, 8, DV)), cu, start, cached_keys(seed, 25, (B, RING, 8, DQK)),
+                  bf16_normal(seed, 26, (B, RING, 8, DV)), name=f"swa_verify_b{B}_q{q_len}")
+    return glb, swa
+
+
 def sample_rows(seed: int, n_total: int, n_sample: int, always=()) -> np.ndarray:
     always = [r for r in always if 0 <= r < n_total]
     perm = synth.permutation(synth.stream_seed(seed, 99), n_total)
