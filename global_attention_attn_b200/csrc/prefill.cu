@@ -620,7 +620,9 @@ struct SwaLayout {
   static constexpr int kOffSink = kOffSeq + 6 * (kMaxSeqs + 1) * 4;
   static constexpr int kOffCS = (kOffSink + 64 * 4 + 1023) / 1024 * 1024;  // float2 [2][R][32] per Q stage (TMA)
   static constexpr int kCSStage = C::R * 32 * 8;
-  static constexpr int kBytes = kOffCS + 2 * kCSStage;
+  static constexpr int kOffStage = kOffCS + 2 * kCSStage;  // O staging: 8 softmax warps x 32 rows x 64 bytes
+  static constexpr int kStageBytes = 32 * 64;
+  static constexpr int kBytes = kOffStage + 8 * kStageBytes;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory budget");
   static_assert(kOffCS % 128 == 0 && kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
@@ -1056,8 +1058,12 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
       if (!wait_w(pv_done(b), ph)) break;
       tc_fence_after();
       const float sc = p.v_scale / l_row;
-      uint16_t* orow = p.out + (long(T.q_row0 + r) * kHq + head) * kDv;
       {
+        // O rows go out through a per-warp staging buffer, 32 columns at a time: each
+        // thread writes its row's 64 bytes (16-byte units XOR-swizzled by row pair), then
+        // a store instruction writes 64 contiguous bytes of each of 8 rows (one position,
+        // the 8 heads) instead of 16 bytes of each of 32 rows.
+        uint8_t* stage = smem + Ly::kOffStage + (warp - 2) * Ly::kStageBytes;
         const uint64_t sc2 = pack_f32x2(sc, sc);
         uint32_t oa[32], ob[32];
         auto store_chunk = [&](uint32_t* o, int c) {
@@ -1066,11 +1072,20 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
             const uint64_t t = mul_f32x2(pack_f32x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), sc2);
             o[i] = pack_bf16x2(lo_f32(t), hi_f32(t));
           }
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(stage + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rho = 8 * k + (lane >> 2), u = lane & 3;  // warp row (position quad*4 + k, head rho % 8)
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + rho * 64 + ((u ^ ((rho >> 1) & 3)) << 4));
+            if (quad * 4 + k < T.rows_valid)
+              *reinterpret_cast<uint4*>(p.out + (long(T.q_row0 + quad * 4 + k) * kHq + T.g * G + (lane >> 2)) * kDv +
+                                        c + 8 * u) = v;
           }
+          __syncwarp();
         };
         tmem_ld32(t_lane + kSwaColO, oa);
         tmem_wait_ld_r32(oa);
