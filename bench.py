@@ -73,7 +73,8 @@ def decode_counts(cfg):
     vis = np.minimum(cfg.ctx, L.window) if L.window else cfg.ctx
     keys = int(vis.astype(np.int64).sum())
     B = len(cfg.ctx)
-    by = keys * L.num_kv_heads * (192 + 128) * 2 + B * 64 * (192 * 2 + 128 * 2 + 4) + B * 4
+    esize = 1 if getattr(cfg, "cache_dtype", 0) == 1 else 2  # E4M3 or bf16 cache elements
+    by = keys * L.num_kv_heads * (192 + 128) * esize + B * 64 * (192 * 2 + 128 * 2 + 4) + B * 4
     if cfg.paged:
         by += int(((cfg.ctx + 127) // 128).sum()) * 4
     return keys * 64 * FLOP_PER_PAIR, by
@@ -255,7 +256,13 @@ class Decode:
         self.cfg, self.M = cfg, M
         L = cfg.layer
         self.q, self.ctx = dev_bf16(cfg.q), dev_i32(cfg.ctx)
-        self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
+        self.fp8 = {}
+        if cfg.cache_dtype == M.MIMO_DTYPE_FP8_E4M3:
+            self.kc = torch.from_numpy(np.ascontiguousarray(cfg.k_cache)).cuda()
+            self.vc = torch.from_numpy(np.ascontiguousarray(cfg.v_cache)).cuda()
+            self.fp8 = dict(cache_dtype=cfg.cache_dtype, k_dequant=dev_f32(cfg.k_dequant), v_dequant=dev_f32(cfg.v_dequant))
+        else:
+            self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
         self.sink = dev_f32(L.sink)
         self.extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
                           num_pages=cfg.k_cache.shape[0]) if cfg.paged else dict(cache_kind=M.MIMO_CACHE_RING)
@@ -270,7 +277,7 @@ class Decode:
         self.M.mimo_attn_decode(self.q, self.ctx, max_seq_len=int(self.cfg.ctx.max()), num_kv_heads=L.num_kv_heads,
                                 rope_base=L.rope_base, window=L.window, k_cache=self.kc, v_cache=self.vc,
                                 sink=self.sink, out=self.out, lse=self.lse, workspace=self.ws,
-                                kernel_events=kernel_events, **self.extra)
+                                kernel_events=kernel_events, **self.extra, **self.fp8)
 
 
 class Chunked:
@@ -404,7 +411,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--main-only", action="store_true", help="skip the per-config details and the CPU baseline")
-    ap.add_argument("--profile", choices=["swa", "global", "decode"],
+    ap.add_argument("--profile", choices=["swa", "global", "decode", "decode_fp8"],
                     help="run only a small case of one kernel (inputs > L2, < 1 GB on the device) for ncu captures")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
@@ -535,6 +542,16 @@ def main():
             e["GB/s"] = bd / (td * 1e-3) / 1e9
             per[name] = e
             del w
+        # the same global decode over an E4M3 cache (per-KV-head scales)
+        c8 = configs.decode_fp8(ctx=gl.ctx)
+        fd, bd = decode_counts(c8)
+        w = Decode(c8)
+        for _ in range(3):
+            w()
+        td = event_time_ms(w, 20) / 20
+        per["global_decode_b64_paged128_fp8"] = _entry(fd, bd, td, hbm, tf_burst, "inputs larger than L2")
+        del w, c8
+        torch.cuda.empty_cache()
         # speculative verification: 4 draft tokens per sequence on the config-3 caches
         vg, vs = configs.verify(B=64, q_len=4, decode=gl)
         for name, c in (("global_verify_b64_q4", vg), ("swa_verify_b64_q4", vs)):
@@ -577,6 +594,8 @@ def profile_case(name):
                                        configs.bf16_normal(5, 3, (T, 8, 128)), cu, cu.copy(), name="swa_prefill_2x4096"))
     if name == "global":
         return Prefill(configs.config2(S=4096))
+    if name == "decode_fp8":
+        return Decode(configs.decode_fp8(B=16))
     sw, gl = configs.config3(B=16)
     return Decode(gl)
 

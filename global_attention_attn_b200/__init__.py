@@ -25,6 +25,8 @@ MIMO_STATUS_BAD_INDEX = 2
 MIMO_CACHE_NONE = 0
 MIMO_CACHE_PAGED = 1
 MIMO_CACHE_RING = 2
+MIMO_DTYPE_BF16 = 0
+MIMO_DTYPE_FP8_E4M3 = 1
 
 NUM_Q_HEADS = 64
 HEAD_DIM_QK = 192
@@ -61,7 +63,7 @@ class MimoDecodeArgs(C.Structure):
                 ("seq_lens", _P), ("cache_kind", C.c_int), ("k_cache", _P), ("v_cache", _P),
                 ("block_table", _P), ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P),
                 ("workspace", _P), ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P),
-                ("ev_kernel_end", _P)]
+                ("ev_kernel_end", _P), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P)]
 
 
 class MimoAppendArgs(C.Structure):
@@ -69,7 +71,7 @@ class MimoAppendArgs(C.Structure):
                 ("head_dim_v", C.c_int), ("rope_dim", C.c_int), ("rope_base", C.c_double), ("k_new", _P),
                 ("v_new", _P), ("pos", _P), ("seq_idx", _P), ("cache_kind", C.c_int), ("k_cache", _P),
                 ("v_cache", _P), ("num_seqs", C.c_int), ("block_table", _P), ("max_pages", C.c_int),
-                ("num_pages", C.c_int)]
+                ("num_pages", C.c_int), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P)]
 
 
 _lib = None
@@ -194,7 +196,8 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
 def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_base: float, window: int,
                      cache_kind: int, k_cache, v_cache, block_table=None, num_pages: int = 0, sink=None, out=None,
                      lse=None, workspace=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE,
-                     stream=None, with_lse: bool = True, kernel_events=None):
+                     stream=None, with_lse: bool = True, kernel_events=None, cache_dtype: int = MIMO_DTYPE_BF16,
+                     k_dequant=None, v_dequant=None):
     """Decode step (see include/mimoattn.h).  kernel_events as for mimo_attn_prefill (around the
     split kernel, not the combine).  Returns (out, lse)."""
     import torch
@@ -218,13 +221,15 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
+    a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
     _check(lib().mimo_attn_decode(C.byref(a), _stream(stream)))
     return out, lse
 
 
 def mimo_attn_decode_noalloc(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_base: float, window: int,
                              cache_kind: int, k_cache, v_cache, out, lse=None, block_table=None, num_pages: int = 0,
-                             sink=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None):
+                             sink=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None,
+                             cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None):
     """Decode that allocates nothing (see mimo_attn_decode_noalloc in include/mimoattn.h): the
     caller passes the output buffers; the split-KV partials go to the library's static
     device scratch (16 MiB), so concurrent calls must not overlap on the GPU."""
@@ -237,13 +242,16 @@ def mimo_attn_decode_noalloc(q, seq_lens, *, max_seq_len: int, num_kv_heads: int
     a.max_pages = 0 if block_table is None else block_table.shape[1]
     a.num_pages = num_pages
     a.out, a.lse = _ptr(out), _ptr(lse)
+    a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
     _check(lib().mimo_attn_decode_noalloc(C.byref(a), _stream(stream)))
     return out, lse
 
 
 def mimo_kv_append(k_new, v_new, pos, seq_idx, *, rope_base: float, cache_kind: int, k_cache, v_cache,
-                   num_seqs: int, block_table=None, num_pages: int = 0, stream=None):
-    """Rotate and store new keys/values into the ring or paged cache (see include/mimoattn.h)."""
+                   num_seqs: int, block_table=None, num_pages: int = 0, stream=None,
+                   cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None):
+    """Rotate and store new keys/values into the ring or paged cache (see include/mimoattn.h);
+    an E4M3 cache (cache_dtype) quantises with the per-KV-head scales k_dequant / v_dequant."""
     a = MimoAppendArgs()
     a.num_tokens, a.num_kv_heads = k_new.shape[0], k_new.shape[1]
     a.head_dim_qk, a.head_dim_v, a.rope_dim, a.rope_base = HEAD_DIM_QK, HEAD_DIM_V, ROPE_DIM, float(rope_base)
@@ -254,6 +262,7 @@ def mimo_kv_append(k_new, v_new, pos, seq_idx, *, rope_base: float, cache_kind: 
     a.block_table = _ptr(block_table)
     a.max_pages = 0 if block_table is None else block_table.shape[1]
     a.num_pages = num_pages
+    a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
     _check(lib().mimo_kv_append(C.byref(a), _stream(stream)))
 
 

@@ -107,14 +107,29 @@ int get_encoder(const char* fn, EncodeTiledFn* out) {
 
 // 3-D bf16 tensor [rows, heads, dim] (dim innermost) with box {64, box_h, box_rows},
 // 128-byte swizzle, zero fill out of bounds.
+int check_cache_dtype(const char* fn, int dtype, const float* kdq, const float* vdq) {
+  if (dtype != MIMO_DTYPE_BF16 && dtype != MIMO_DTYPE_FP8_E4M3)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: unknown cache_dtype %d", fn, dtype);
+  if (dtype == MIMO_DTYPE_FP8_E4M3) {
+    if (!kdq || !vdq) return fail(MIMO_ERR_INVALID_ARG, "%s: an E4M3 cache needs k_dequant and v_dequant", fn);
+    if ((reinterpret_cast<uintptr_t>(kdq) | reinterpret_cast<uintptr_t>(vdq)) & 3)
+      return fail(MIMO_ERR_INVALID_ARG, "%s: k_dequant / v_dequant are not 4-byte aligned", fn);
+  }
+  return MIMO_OK;
+}
+
+// 3-D map [rows, heads, dim] with boxes of 64 elements x box_h heads x box_rows rows:
+// bf16 with the 128-byte swizzle, or (fp8) one-byte elements with the 64-byte swizzle.
 int make_map(const char* fn, EncodeTiledFn enc, CUtensorMap* m, const void* base, long rows, int heads, int dim,
-             int box_h, int box_rows) {
+             int box_h, int box_rows, bool fp8 = false) {
+  const cuuint64_t es = fp8 ? 1 : 2;
   cuuint64_t gdim[3] = {cuuint64_t(dim), cuuint64_t(heads), cuuint64_t(rows < 1 ? 1 : rows)};
-  cuuint64_t gstride[2] = {cuuint64_t(dim) * 2, cuuint64_t(dim) * 2 * heads};
+  cuuint64_t gstride[2] = {cuuint64_t(dim) * es, cuuint64_t(dim) * es * heads};
   cuuint32_t box[3] = {64, cuuint32_t(box_h), cuuint32_t(box_rows)};
   cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MIMO_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", fn, int(r));
   return MIMO_OK;
@@ -187,6 +202,7 @@ int mimo_kv_append(const mimo_append_args* a, void* stream) {
     if (a->max_pages <= 0 || a->num_pages <= 0)
       return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages and num_pages must be > 0 for a paged cache", fn);
   }
+  if (int rc = check_cache_dtype(fn, a->cache_dtype, a->k_dequant, a->v_dequant)) return rc;
   DevState d;
   if (int rc = dev_state(fn, &d)) return rc;
   AppendParams p;
@@ -203,6 +219,9 @@ int mimo_kv_append(const mimo_append_args* a, void* stream) {
   p.block_table = a->block_table;
   p.max_pages = a->max_pages;
   p.num_pages = a->num_pages;
+  p.fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
+  p.k_dequant = a->k_dequant;
+  p.v_dequant = a->v_dequant;
   p.rope = make_freqs(a->rope_base);
   p.status = d.status;
   cudaError_t e = launch_kv_append(p, static_cast<cudaStream_t>(stream));
@@ -235,6 +254,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
     if (long(a->max_pages) * kPage < a->max_seq_len)
       return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages * 128 is below max_seq_len", fn);
   }
+  if (int rc = check_cache_dtype(fn, a->cache_dtype, a->k_dequant, a->v_dequant)) return rc;
   const size_t need = mimo_attn_decode_workspace_size(a->batch, a->max_seq_len, a->layer.num_kv_heads, a->layer.window);
   if (need > 0) {
     if (!a->workspace || a->workspace_bytes < need)
@@ -250,9 +270,10 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   std::memset(&p, 0, sizeof(p));
   {
     const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * kPage : long(a->num_pages) * kPage;
+    const bool fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
     int rc = make_map(fn, enc, &p.tm_q, a->q, a->batch, kHq, kDqk, 16, 1);
-    if (!rc) rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 16);
-    if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 16);
+    if (!rc) rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 16, fp8);
+    if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 16, fp8);
     if (rc) return rc;
   }
   p.batch = a->batch;
@@ -279,6 +300,9 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   p.ws_ml = need ? reinterpret_cast<float*>(static_cast<char*>(a->workspace) +
                                             round256(size_t(a->batch) * kHq * p.max_splits * kDv * 4))
                  : nullptr;
+  p.fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
+  p.k_dequant = a->k_dequant;
+  p.v_dequant = a->v_dequant;
   p.rope = make_freqs(a->layer.rope_base);
   p.status = d.status;
   cudaError_t e = launch_decode(p, d.sms, static_cast<cudaStream_t>(stream), a->ev_kernel_begin, a->ev_kernel_end);

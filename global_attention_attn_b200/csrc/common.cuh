@@ -33,6 +33,21 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
   sincosf(r, s, c);
 }
 
+// OCP E4M3 (FP8) conversions.  Two floats -> two E4M3 bytes (round to nearest even,
+// saturating to +-448): `lo` lands in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// Two E4M3 bytes -> two fp16 (exact: E4M3 is a subset of fp16); the low byte lands in
+// the low half.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t x) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(x));
+  return d;
+}
+
 // NeoX rotate-half on one 16-byte chunk pair: lo holds dims 8u..8u+7, hi holds
 // dims 8u+32..8u+39 (u in 0..3); frequency index of element i is 8u+i.
 // Input bf16, output IEEE fp16: the rotated dims are kept in fp16 everywhere

@@ -35,21 +35,29 @@ namespace {
 constexpr int kPairs = 4;                      // producer / consumer warp pairs per CTA
 constexpr int kThreads = 2 * kPairs * 32;      // warps 0..3 produce, 4..7 consume
 constexpr int kTileK = 16;                     // keys per TMA tile
-constexpr int kStages = 4;
-constexpr int kChunk = kTileK * 128;           // 16 keys x 64 dims x 2 bytes
-constexpr int kStageBytes = 5 * kChunk;        // K (3 chunks of 64 dims) + V (2 chunks)
 constexpr int kQChunk = 16 * 128;              // 16 heads x 64 dims x 2 bytes
 constexpr int kQBytes = 3 * kQChunk;
-constexpr int kPairBytes = kStages * kStageBytes + 2 * kQBytes;
 constexpr int kInfoBytes = 32 + 32 * 8;        // unit fields + 32 (cos, sin) pairs
-constexpr int kOffInfo = kPairs * kPairBytes;
-constexpr int kOffBar = kOffInfo + kPairs * 2 * kInfoBytes;
-constexpr int kBarsPerPair = 2 * kStages + 4;  // full, empty, q_full[2], q_empty[2]
-constexpr int kOffTbl = kOffBar + kPairs * kBarsPerPair * 8 + 16;
 constexpr int kMaxTable = 1024;                // sequences of the ordered split enumeration
-constexpr int kSmemBytes = kOffTbl + 2 * (kMaxTable + 1) * 4 + 1024;
-static_assert(kPairBytes % 1024 == 0 && kStageBytes % 1024 == 0 && kQBytes % 1024 == 0, "swizzle alignment");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Shared memory of one CTA.  A stage holds one 16-key tile: K as three 64-element
+// chunks, V as two; bf16 rows are 128 bytes (128-byte swizzle), E4M3 rows 64 bytes
+// (64-byte swizzle, twice the stages for the same bytes in flight).
+template <bool FP8>
+struct DecodeLayout {
+  static constexpr int kRowBytes = FP8 ? 64 : 128;
+  static constexpr int kChunk = kTileK * kRowBytes;
+  static constexpr int kStageBytes = 5 * kChunk;
+  static constexpr int kStages = FP8 ? 8 : 4;
+  static constexpr int kPairBytes = kStages * kStageBytes + 2 * kQBytes;
+  static constexpr int kOffInfo = kPairs * kPairBytes;
+  static constexpr int kOffBar = kOffInfo + kPairs * 2 * kInfoBytes;
+  static constexpr int kBarsPerPair = 2 * kStages + 4;  // full, empty, q_full[2], q_empty[2]
+  static constexpr int kOffTbl = kOffBar + kPairs * kBarsPerPair * 8 + 16;
+  static constexpr int kSmemBytes = kOffTbl + 2 * (kMaxTable + 1) * 4 + 1024;
+  static_assert(kPairBytes % 1024 == 0 && kStageBytes % 1024 == 0 && kQBytes % 1024 == 0, "swizzle alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -151,7 +159,12 @@ __device__ __forceinline__ void unit_ordered(const DecodeParams& p, const int* t
 
 }  // namespace
 
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+  using Ly = DecodeLayout<FP8>;
+  constexpr int kStages = Ly::kStages, kStageBytes = Ly::kStageBytes, kChunk = Ly::kChunk;
+  constexpr int kPairBytes = Ly::kPairBytes, kOffInfo = Ly::kOffInfo, kOffBar = Ly::kOffBar;
+  constexpr int kBarsPerPair = Ly::kBarsPerPair, kOffTbl = Ly::kOffTbl;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -303,7 +316,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
   // ------------------------------------------------------------ consumer warp
   const int q4 = lane & 3, r0 = lane >> 2, r1 = r0 + 8;
-  const float c_log2 = p.scale_log2;
   int it = 0;
   for (int n = 0;; ++n) {
     const int b = n & 1;
@@ -315,8 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               t0 = I->t0;
     // ---- query fragments (A of m16n8k16) from the swizzled tile; rows = heads of the group
     uint32_t qa[12][4];
-    {
-      const uint32_t qt = qtile0 + b * kQBytes;
+    const float4* cs = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(I + 1));
+    const uint32_t qt = qtile0 + b * kQBytes;
+    if constexpr (!FP8) {
       const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < 12; ++kk) {
@@ -324,7 +337,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         ldsm_x4(qt + (kk >> 2) * kQChunk + row * 128 + unit16 * 16, qa[kk]);
       }
       // dims j < 32 (k-steps 0, 1) pair with dims j + 32 (k-steps 2, 3) in the same register slot
-      const float4* cs = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(I + 1));
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
@@ -336,9 +348,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           qa[kk][e] = pack2_f16(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
           qa[kk + 2][e] = pack2_f16(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
         }
+    } else {
+      // E4M3 keys are read with ldmatrix as pairs of bytes, which gives thread (r0, q4) the
+      // 4 consecutive dims 4q4..4q4+3 of a 16-dim step: the step's k order is permuted the
+      // same way here (k 2q4, 2q4+1 <- dims 4q4, 4q4+1; k 2q4+8, 2q4+9 <- dims 4q4+2, 4q4+3),
+      // which leaves the dot products unchanged.  Everything runs in fp16.
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk) {
+        const int unit16 = 2 * (kk & 3) + (q4 >> 1);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = hf ? r1 : r0;
+          const uint2 w = *reinterpret_cast<const uint2*>(smem + (qt - sbase) + (kk >> 2) * kQChunk + row * 128 +
+                                                          ((unit16 ^ (row & 7)) << 4) + 8 * (q4 & 1));
+          qa[kk][hf] = w.x;      // dims 4q4, 4q4 + 1 of the step
+          qa[kk][2 + hf] = w.y;  // dims 4q4 + 2, 4q4 + 3
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = 16 * kk + 4 * q4 + ((e & 2) ? 2 : 0);
+          const float4 t = cs[j0 >> 1];
+          const uint32_t xw = qa[kk][e], yw = qa[kk + 2][e];
+          const float x0 = lo_bf16(xw), x1 = hi_bf16(xw), y0 = lo_bf16(yw), y1 = hi_bf16(yw);
+          qa[kk][e] = pack2_f16(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
+          qa[kk + 2][e] = pack2_f16(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+        }
+#pragma unroll
+      for (int kk = 4; kk < 12; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qa[kk][e] = pack2_f16(lo_bf16(qa[kk][e]), hi_bf16(qa[kk][e]));
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(q_empty(b));
+    const float c_log2 = FP8 ? p.scale_log2 * p.k_dequant[g] : p.scale_log2;
+    const float v_deq = FP8 ? p.v_dequant[g] : 1.f;
 
     float m_r[2] = {-INFINITY, -INFINITY};
     float l_r[2] = {0.f, 0.f};
@@ -355,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       float acc[4][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-      {
+      if constexpr (!FP8) {
         // B fragments of K^T: matrices (keys 0-7 | 8-15) x (dims lo 8 | hi 8);
         // rows are 128-byte swizzled (16-byte unit u of row k sits at u ^ (k & 7))
         const int key = (lane & 7) + (lane >> 4) * 8;
@@ -373,6 +419,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           } else {
             mma_bf16(a0, qa[kk], bf[0], bf[1]);
             mma_bf16(a1, qa[kk], bf[2], bf[3]);
+          }
+        }
+      } else {
+        // matrices (keys 0-7 | 8-15) x (dims 0-15 | 16-31) of a 32-dim group, 64-byte rows
+        // swizzled by the 64-byte pattern (16-byte unit u of row k sits at u ^ ((k >> 1) & 3))
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int g32 = 0; g32 < 6; ++g32) {
+          const int unit16 = 2 * (g32 & 1) + (lane >> 4);
+          uint32_t bf[4];
+          ldsm_x4(kb + (g32 >> 1) * kChunk + key * 64 + ((unit16 ^ ((key >> 1) & 3)) << 4), bf);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int kk = 2 * g32 + hf;
+            const uint32_t m_lo = bf[2 * hf], m_hi = bf[2 * hf + 1];  // keys 0-7, keys 8-15
+            mma_f16(acc[kk & 1], qa[kk], f16x2_from_e4m3x2(uint16_t(m_lo)), f16x2_from_e4m3x2(uint16_t(m_lo >> 16)));
+            mma_f16(acc[2 + (kk & 1)], qa[kk], f16x2_from_e4m3x2(uint16_t(m_hi)),
+                    f16x2_from_e4m3x2(uint16_t(m_hi >> 16)));
           }
         }
       }
@@ -432,11 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         o[i][3] *= al1;
       }
       uint32_t pa[4];
-      pa[0] = pack2_bf16(p0[0], p0[1]);
-      pa[1] = pack2_bf16(p0[2], p0[3]);
-      pa[2] = pack2_bf16(p1[0], p1[1]);
-      pa[3] = pack2_bf16(p1[2], p1[3]);
-      {
+      if constexpr (!FP8) {
+        pa[0] = pack2_bf16(p0[0], p0[1]);
+        pa[1] = pack2_bf16(p0[2], p0[3]);
+        pa[2] = pack2_bf16(p1[0], p1[1]);
+        pa[3] = pack2_bf16(p1[2], p1[3]);
         // B fragments of V (trans): matrices (keys 0-7 | 8-15) x (dims d0 .. d0+7 | d0+8 ..)
         const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
         const int dq = lane >> 4;
@@ -447,6 +511,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           ldsm_x4_t(vb + (n2 >> 2) * kChunk + key * 128 + unit16 * 16, bf);
           mma_bf16(o[2 * n2], pa, bf[0], bf[1]);
           mma_bf16(o[2 * n2 + 1], pa, bf[2], bf[3]);
+        }
+      } else {
+        pa[0] = pack2_f16(p0[0], p0[1]);
+        pa[1] = pack2_f16(p0[2], p0[3]);
+        pa[2] = pack2_f16(p1[0], p1[1]);
+        pa[3] = pack2_f16(p1[2], p1[3]);
+        // Transposed byte-pair matrices (keys 0-7 | 8-15) x (dims of a 16-dim block): a
+        // thread gets dims 2r0, 2r0+1 of keys 2q4, 2q4+1; the even and the odd dim make
+        // two n8 blocks of the PV product.  o[2B] holds dims 16B + 4q4 + {0, 2}, o[2B+1]
+        // dims 16B + 4q4 + {1, 3}.
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int h32 = 0; h32 < 4; ++h32) {
+          const int unit16 = 2 * (h32 & 1) + (lane >> 4);
+          uint32_t bf[4];
+          ldsm_x4_t(vb + (h32 >> 1) * kChunk + key * 64 + ((unit16 ^ ((key >> 1) & 3)) << 4), bf);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int blk = 2 * h32 + hf;
+            const uint32_t m_lo = bf[2 * hf], m_hi = bf[2 * hf + 1];  // keys 0-7, keys 8-15
+            mma_f16(o[2 * blk], pa, f16x2_from_e4m3x2(uint16_t(__byte_perm(m_lo, 0, 0x0020))),
+                    f16x2_from_e4m3x2(uint16_t(__byte_perm(m_hi, 0, 0x0020))));
+            mma_f16(o[2 * blk + 1], pa, f16x2_from_e4m3x2(uint16_t(__byte_perm(m_lo, 0, 0x0031))),
+                    f16x2_from_e4m3x2(uint16_t(__byte_perm(m_hi, 0, 0x0031))));
+          }
         }
       }
       __syncwarp();
@@ -473,16 +562,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           f = ex2(M - M2);
           L2 = L * f + ex2(sl - M2);
         }
-        const float sc = p.v_scale * f / L2;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (long(s) * kHq + h) * kDv + 2 * q4);
+        const float sc = p.v_scale * f / L2 * v_deq;
+        if constexpr (!FP8) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (long(s) * kHq + h) * kDv + 2 * q4);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i * 4] = pack2_bf16(o[i][2 * half] * sc, o[i][2 * half + 1] * sc);
+          for (int i = 0; i < 16; ++i) dst[i * 4] = pack2_bf16(o[i][2 * half] * sc, o[i][2 * half + 1] * sc);
+        } else {
+          uint2* dst = reinterpret_cast<uint2*>(p.out + (long(s) * kHq + h) * kDv + 4 * q4);
+#pragma unroll
+          for (int blk = 0; blk < 8; ++blk)
+            dst[4 * blk] = make_uint2(pack2_bf16(o[2 * blk][2 * half] * sc, o[2 * blk + 1][2 * half] * sc),
+                                      pack2_bf16(o[2 * blk][2 * half + 1] * sc, o[2 * blk + 1][2 * half + 1] * sc));
+        }
         if (p.lse && q4 == 0) p.lse[long(s) * kHq + h] = (M2 + __log2f(L2)) * kLn2;
       } else {
-        float* dst = p.ws_o + ((long(s) * kHq + h) * p.max_splits + split) * kDv + 2 * q4;
+        float* dst = p.ws_o + ((long(s) * kHq + h) * p.max_splits + split) * kDv;
+        if constexpr (!FP8) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          *reinterpret_cast<float2*>(dst + i * 8) = make_float2(o[i][2 * half], o[i][2 * half + 1]);
+          for (int i = 0; i < 16; ++i)
+            *reinterpret_cast<float2*>(dst + i * 8 + 2 * q4) = make_float2(o[i][2 * half], o[i][2 * half + 1]);
+        } else {
+#pragma unroll
+          for (int blk = 0; blk < 8; ++blk)
+            *reinterpret_cast<float4*>(dst + 16 * blk + 4 * q4) =
+                make_float4(o[2 * blk][2 * half] * v_deq, o[2 * blk + 1][2 * half] * v_deq,
+                            o[2 * blk][2 * half + 1] * v_deq, o[2 * blk + 1][2 * half + 1] * v_deq);
+        }
         if (q4 == 0) {
           float* ml = p.ws_ml + ((long(s) * kHq + h) * p.max_splits + split) * 2;
           ml[0] = M;
@@ -541,15 +646,22 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const __grid_consta
   if (p.lse && lane == 0) p.lse[long(s) * kHq + h] = (M + __log2f(L)) * kLn2;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* ev_begin, void* ev_end) {
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+template <bool FP8>
+cudaError_t launch_decode_kernel(const DecodeParams& p, int grid, cudaStream_t s) {
+  using Ly = DecodeLayout<FP8>;
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kSmemBytes);
   if (e != cudaSuccess) return e;
+  decode_kernel<FP8><<<grid, kThreads, Ly::kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* ev_begin, void* ev_end) {
   const long units = long(p.batch) * p.hkv * p.max_splits;
   const long ctas = (units + kPairs - 1) / kPairs;
   const int grid = int(ctas < sms ? ctas : sms);
+  cudaError_t e;
   if (ev_begin && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s)) != cudaSuccess) return e;
-  decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
-  e = cudaGetLastError();
+  e = p.fp8 ? launch_decode_kernel<true>(p, grid, s) : launch_decode_kernel<false>(p, grid, s);
   if (e != cudaSuccess) return e;
   if (ev_end && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s)) != cudaSuccess) return e;
   if (p.max_splits <= 1) return e;

@@ -31,6 +31,9 @@ struct AppendParams {
   int num_seqs;
   const int32_t* block_table;
   int max_pages, num_pages;
+  int fp8;                   // cache rows hold E4M3 bytes (quantised by 1 / k_dequant[g], 1 / v_dequant[g])
+  const float* k_dequant;
+  const float* v_dequant;
   RopeFreqs rope;
   unsigned* status;
 };
@@ -56,6 +59,9 @@ struct DecodeParams {
   float* lse;
   float* ws_o;   // [batch, 64, max_splits, 128]
   float* ws_ml;  // [batch, 64, max_splits, 2]
+  int fp8;                   // E4M3 cache rows with per-KV-head dequantisation scales
+  const float* k_dequant;
+  const float* v_dequant;
   RopeFreqs rope;
   unsigned* status;
 };

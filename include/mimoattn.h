@@ -78,6 +78,20 @@ typedef struct {
 #define MIMO_CACHE_PAGED 1 /* [num_pages, 128, Hkv, D] pages of 128 positions, via block_table */
 #define MIMO_CACHE_RING 2  /* [num_seqs, 128, Hkv, D]: position p of sequence s in slot p % 128 */
 
+/* Cache element formats (mimo_decode_args.cache_dtype, mimo_append_args.cache_dtype).
+ *   MIMO_DTYPE_BF16: key dims 0..63 (the rotated part) as IEEE fp16, key dims
+ *     64..191 and the value as bf16 (2 bytes per element).
+ *   MIMO_DTYPE_FP8_E4M3: every key and value element is one OCP E4M3 byte; it
+ *     stands for code * k_dequant[g] (keys of KV head g) or code * v_dequant[g]
+ *     (values).  Appends quantise x / dequant with round-to-nearest-even,
+ *     saturating at +-448.  Decode only (prefill reads bf16 caches).  The vLLM
+ *     recipe page for MiMo-V2.6-Flash ("Launch command", the AMD MI355X line)
+ *     serves the model with an FP8 KV cache (--kv-cache-dtype fp8) without
+ *     saying how it is scaled; one scale per KV head is this library's reading.
+ *     It halves the bytes a decode step streams. */
+#define MIMO_DTYPE_BF16 0
+#define MIMO_DTYPE_FP8_E4M3 1
+
 /*
  * Prefill (varlen, causal, window or global, sink on/off).
  *
@@ -172,6 +186,9 @@ typedef struct {
    * cudaEventElapsedTime gives that kernel's device time. */
   void* ev_kernel_begin;
   void* ev_kernel_end;
+  int cache_dtype;          /* MIMO_DTYPE_BF16 (default 0) or MIMO_DTYPE_FP8_E4M3 */
+  const float* k_dequant;   /* FP8: device fp32 [num_kv_heads] key scales, else NULL */
+  const float* v_dequant;   /* FP8: device fp32 [num_kv_heads] value scales, else NULL */
 } mimo_decode_args;
 
 /* Bytes of workspace mimo_attn_decode needs (split-KV partials). */
@@ -232,6 +249,9 @@ typedef struct {
   const int32_t* block_table; /* paged: device int32 [num_seqs, max_pages] */
   int max_pages;
   int num_pages;
+  int cache_dtype;          /* MIMO_DTYPE_BF16 (default 0) or MIMO_DTYPE_FP8_E4M3 */
+  const float* k_dequant;   /* FP8: device fp32 [num_kv_heads], else NULL */
+  const float* v_dequant;
 } mimo_append_args;
 
 MIMO_API int mimo_kv_append(const mimo_append_args* args, void* stream);

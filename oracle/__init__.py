@@ -36,6 +36,7 @@ class OracleLayer(C.Structure):
         ("k_new", P_U16), ("v_new", P_U16), ("new_row0", P_I32), ("new_pos0", P_I32), ("new_len", P_I32),
         ("cache_kind", C.c_int), ("k_cache", P_U16), ("v_cache", P_U16), ("page_size", C.c_int),
         ("block_table", P_I32), ("max_pages", C.c_int),
+        ("cache_dtype", C.c_int), ("k_dequant", P_F32), ("v_dequant", P_F32),
     ]
 
 
@@ -62,6 +63,8 @@ def lib():
         _lib.oracle_kv_append.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, P_U16, P_U16,
                                           P_I32, P_F64, P_F64]
         _lib.oracle_kv_append.restype = C.c_int
+        _lib.oracle_e4m3_to_double.argtypes = [C.c_int]
+        _lib.oracle_e4m3_to_double.restype = C.c_double
     return _lib
 
 
@@ -85,8 +88,9 @@ def attention(*, q, hq, hkv, dqk, dv, rope_dim, rope_base, softmax_scale, v_scal
               q_row0, q_len, q_pos0, sel_seq, sel_row,
               k_new=None, v_new=None, new_row0=None, new_pos0=None, new_len=None,
               cache_kind=0, k_cache=None, v_cache=None, page_size=0, block_table=None,
-              nthreads=None, online=False):
+              cache_dtype=0, k_dequant=None, v_dequant=None, nthreads=None, online=False):
     """Evaluates the selected rows (sel_seq[i], row sel_row[i] of that sequence) for all heads.
+    cache_dtype 1: the caches hold E4M3 bytes with per-KV-head scales k_dequant / v_dequant.
 
     Returns (out [n, hq, dv] float64, lse [n, hq] float64)."""
     keep = []
@@ -114,8 +118,12 @@ def attention(*, q, hq, hkv, dqk, dv, rope_dim, rope_base, softmax_scale, v_scal
     L.new_pos0 = _ptr(arr(new_pos0 if new_pos0 is not None else zeros, np.int32), P_I32)
     L.new_len = _ptr(arr(new_len if new_len is not None else zeros, np.int32), P_I32)
     L.cache_kind = int(cache_kind)
-    L.k_cache = _ptr(arr(k_cache, np.uint16), P_U16)
-    L.v_cache = _ptr(arr(v_cache, np.uint16), P_U16)
+    cdt = np.uint8 if cache_dtype == 1 else np.uint16
+    L.k_cache = C.cast(_ptr(arr(k_cache, cdt), C.c_void_p), P_U16) if k_cache is not None else None
+    L.v_cache = C.cast(_ptr(arr(v_cache, cdt), C.c_void_p), P_U16) if v_cache is not None else None
+    L.cache_dtype = int(cache_dtype)
+    L.k_dequant = _ptr(arr(k_dequant, np.float32), P_F32)
+    L.v_dequant = _ptr(arr(v_dequant, np.float32), P_F32)
     L.page_size = int(page_size)
     bt = arr(block_table, np.int32)
     L.block_table = _ptr(bt, P_I32)
@@ -132,6 +140,13 @@ def attention(*, q, hq, hkv, dqk, dv, rope_dim, rope_base, softmax_scale, v_scal
     if rc != 0:
         raise RuntimeError(f"oracle_attention failed with code {rc}")
     return out, lse
+
+
+def e4m3_to_double(codes) -> np.ndarray:
+    """Values of E4M3 bytes (OCP 8-bit floating point), in float64."""
+    codes = np.asarray(codes, np.int64)
+    f = lib().oracle_e4m3_to_double
+    return np.array([f(int(c)) for c in codes.reshape(-1)], np.float64).reshape(codes.shape)
 
 
 def kv_append(k_new, v_new, pos, rope_base: float, rope_dim: int = 64):

@@ -56,9 +56,24 @@ inline double f16_to_double(uint16_t h) {
   return sign ? -v : v;
 }
 
+// OCP 8-bit floating point, E4M3 ("FP8 E4M3"): 1 sign bit, 4 exponent bits
+// (bias 7), 3 mantissa bits; exponent 0 holds zero and the subnormals m/8 * 2^-6;
+// no infinities; exponent 15 with mantissa 7 is NaN, so the largest value is
+// 1.75 * 2^8 = 448.
+inline double e4m3_to_double(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+  double v;
+  if (e == 0) v = std::ldexp(double(m), -9);                        // (m / 8) * 2^-6
+  else if (e == 15 && m == 7) v = NAN;
+  else v = std::ldexp(double(8 + m), e - 10);                        // (1 + m/8) * 2^(e-7)
+  return sign ? -v : v;
+}
+
 }  // namespace
 
 extern "C" {
+
+double oracle_e4m3_to_double(int code) { return e4m3_to_double(uint8_t(code)); }
 
 // Layer description plus where each sequence's keys live.  Keys at positions
 // [new_pos0[s], new_pos0[s] + new_len[s]) come from the contiguous pre-RoPE
@@ -67,7 +82,9 @@ extern "C" {
 //   cache_kind 1 (paged): page block_table[s * max_pages + pos / page_size], slot pos % page_size
 //   cache_kind 2 (ring):  entry s * page_size + pos % page_size
 // Cache rows use the library's cache format: key dims < rope_dim are IEEE
-// fp16 bit patterns (the rotated part), the other key dims and the values bf16.
+// fp16 bit patterns (the rotated part), the other key dims and the values bf16
+// (cache_dtype 0); or every key and value element is an E4M3 byte that
+// dequantises to code * k_dequant[g] (keys) / code * v_dequant[g] (values) (cache_dtype 1).
 typedef struct {
   int hq, hkv, dqk, dv, rope_dim;
   double rope_base, softmax_scale, v_scale;
@@ -88,6 +105,9 @@ typedef struct {
   int page_size;
   const int32_t* block_table;
   int max_pages;
+  int cache_dtype;
+  const float* k_dequant;  // [hkv], cache_dtype 1
+  const float* v_dequant;
 } oracle_layer;
 
 // Partial NeoX rotation of one head vector x[0..d) at position pos, in double.
@@ -137,6 +157,15 @@ bool fetch_key(const Ctx& C, int s, int p, int g, double* k, double* v) {
       entry = size_t(page) * L->page_size + (p % L->page_size);
     } else {
       entry = size_t(s) * L->page_size + (p % L->page_size);
+    }
+    if (L->cache_dtype == 1) {
+      const uint8_t* kp = reinterpret_cast<const uint8_t*>(L->k_cache) + (entry * L->hkv + g) * L->dqk;
+      const uint8_t* vp = reinterpret_cast<const uint8_t*>(L->v_cache) + (entry * L->hkv + g) * L->dv;
+      if (k)
+        for (int i = 0; i < L->dqk; ++i) k[i] = e4m3_to_double(kp[i]) * double(L->k_dequant[g]);
+      if (v)
+        for (int i = 0; i < L->dv; ++i) v[i] = e4m3_to_double(vp[i]) * double(L->v_dequant[g]);
+      return true;
     }
     const uint16_t* kp = L->k_cache + (entry * L->hkv + g) * L->dqk;
     const uint16_t* vp = L->v_cache + (entry * L->hkv + g) * L->dv;

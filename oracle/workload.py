@@ -45,6 +45,7 @@ def decode(cfg, seqs=None, nthreads=None):
     seqs = np.asarray(seqs, np.int32)
     kw = dict(cache_kind=1, page_size=cfg.k_cache.shape[1], block_table=cfg.block_table) if cfg.paged else \
         dict(cache_kind=2, page_size=cfg.k_cache.shape[1])
+    kw.update(cache_dtype=cfg.cache_dtype, k_dequant=cfg.k_dequant, v_dequant=cfg.v_dequant)
     return attention(q=cfg.q, **_layer_kw(cfg.layer), q_row0=np.arange(B, dtype=np.int32),
                      q_len=np.ones(B, np.int32), q_pos0=(cfg.ctx - 1).astype(np.int32), sel_seq=seqs,
                      sel_row=np.zeros(len(seqs), np.int32), new_row0=np.zeros(B, np.int32),

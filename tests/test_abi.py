@@ -147,6 +147,10 @@ def _decode_args(**over):
     ({"workspace_bytes": 64}, M.MIMO_ERR_WORKSPACE),
     ({"layer.head_dim_v": 64}, M.MIMO_ERR_UNSUPPORTED),
     ({"seq_lens": None}, M.MIMO_ERR_INVALID_ARG),
+    ({"cache_dtype": 5}, M.MIMO_ERR_INVALID_ARG),
+    ({"cache_dtype": M.MIMO_DTYPE_FP8_E4M3}, M.MIMO_ERR_INVALID_ARG),     # E4M3 needs dequant scales
+    ({"cache_dtype": M.MIMO_DTYPE_FP8_E4M3, "k_dequant": C.c_void_p(FAKE), "v_dequant": C.c_void_p(FAKE + 2)},
+     M.MIMO_ERR_INVALID_ARG),                                             # misaligned scales
 ])
 def test_decode_validation(over, code):
     a = _decode_args(**over)

@@ -88,6 +88,64 @@ def test_kv_append(kind):
     assert np.all(kcn[~touched] == 0) and np.all(vcn[~touched] == 0)
 
 
+def _e4m3_grid(x):
+    """Spacing of E4M3 values around |x| (subnormal step 2^-9 below 2^-6)."""
+    a = np.maximum(np.abs(x), 2.0 ** -6)
+    return 2.0 ** (np.floor(np.log2(a)) - 3)
+
+
+@pytest.mark.parametrize("kind", ["ring", "paged"])
+def test_kv_append_fp8(kind):
+    """E4M3 append: every stored byte is a nearest E4M3 value of the oracle's (rotated) element
+    divided by its KV head's scale (either neighbour where the element sits within rounding
+    noise of a midpoint), saturated at 448; untouched slots stay zero."""
+    import torch
+    import global_attention_attn_b200 as M
+    n, hkv, base = (300, 8, 1e4) if kind == "ring" else (500, 4, 1e7)
+    k = configs.bf16_normal(43, 1, (n, hkv, 192))
+    v = configs.bf16_normal(43, 2, (n, hkv, 128))
+    # scales small enough that some elements saturate
+    kdq = np.array([0.004, 0.3, 1.0, 2.5, 0.07, 0.5, 1.5, 0.9][:hkv], np.float32)
+    vdq = np.array([0.01, 0.8, 2.0, 0.6, 1.1, 0.25, 3.0, 0.45][:hkv], np.float32)
+    seq = (np.arange(n) % 3).astype(np.int32)
+    pos = (np.arange(n) // 3 + np.array([0, 5, 120000])[seq]).astype(np.int32)
+    extra = dict(cache_dtype=M.MIMO_DTYPE_FP8_E4M3, k_dequant=dev_f32(kdq), v_dequant=dev_f32(vdq))
+    if kind == "ring":
+        kc = torch.zeros((3, 128, hkv, 192), dtype=torch.uint8, device="cuda")
+        vc = torch.zeros((3, 128, hkv, 128), dtype=torch.uint8, device="cuda")
+        M.mimo_kv_append(dev_bf16(k), dev_bf16(v), dev_i32(pos), dev_i32(seq), rope_base=base,
+                         cache_kind=M.MIMO_CACHE_RING, k_cache=kc, v_cache=vc, num_seqs=3, **extra)
+        where = {(int(seq[t]), int(pos[t] % 128)): t for t in range(n)}
+    else:
+        maxp = (int(pos.max()) // 128) + 1
+        bt = (synth.permutation(8, 3 * maxp).reshape(3, maxp)).astype(np.int32)
+        kc = torch.zeros((3 * maxp, 128, hkv, 192), dtype=torch.uint8, device="cuda")
+        vc = torch.zeros((3 * maxp, 128, hkv, 128), dtype=torch.uint8, device="cuda")
+        M.mimo_kv_append(dev_bf16(k), dev_bf16(v), dev_i32(pos), dev_i32(seq), rope_base=base,
+                         cache_kind=M.MIMO_CACHE_PAGED, k_cache=kc, v_cache=vc, num_seqs=3,
+                         block_table=dev_i32(bt), num_pages=3 * maxp, **extra)
+        where = {(int(bt[seq[t], pos[t] // 128]), int(pos[t] % 128)): t for t in range(n)}
+    ko, vo = oracle.kv_append(k, v, pos, base)
+    kb, vb = kc.cpu().numpy(), vc.cpu().numpy()
+    kval, vval = oracle.e4m3_to_double(kb), oracle.e4m3_to_double(vb)
+    touched = np.zeros(kb.shape[:2], bool)
+    slots = list(where.items())
+    for (a, b), t in slots:
+        touched[a, b] = True
+    rows = np.array([t for _, t in slots])
+    ia = np.array([a for (a, _), _ in slots])
+    ib = np.array([b for (_, b), _ in slots])
+    for got, ref, dq in ((kval[ia, ib], ko[rows], kdq), (vval[ia, ib], vo[rows], vdq)):
+        x = ref / dq.astype(np.float64)[None, :, None]
+        sat = np.abs(x) >= 448.0
+        assert np.all(got[sat] == np.sign(x[sat]) * 448.0)
+        err = np.abs(got[~sat] - x[~sat])
+        half = 0.5 * _e4m3_grid(x[~sat])
+        assert np.all(err <= half * (1 + 2.0 ** -10)), float((err / half).max())
+        assert sat.any() or dq is vdq
+    assert np.all(kb[~touched] == 0) and np.all(vb[~touched] == 0)
+
+
 # ----------------------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("ctx_range", [(1, 127), (100, 3000), (4096, 9000)])
@@ -150,6 +208,39 @@ def test_decode_paged_window_unaligned_splits():
         out, lse = decode_cfg(cfg)
         ro, rl = oracle.decode(cfg)
         parity(out, lse, ro, rl, f"paged decode, window {window}")
+
+
+@pytest.mark.parametrize("ring", [False, True])
+def test_decode_fp8_small(ring):
+    """Decode over an E4M3 cache (per-KV-head scales): ring (sliding layer) and paged (global)."""
+    cfg = configs.decode_fp8(seed=810 + ring, B=8, ctx_range=(1, 3000), ring=ring)
+    out, lse = decode_cfg(cfg)
+    ro, rl = oracle.decode(cfg)
+    parity(out, lse, ro, rl, cfg.name)
+
+
+def test_decode_fp8_split_boundaries_and_window():
+    ctx = np.array([1, 127, 128, 129, 511, 512, 513, 1025, 8193], np.int32)
+    cfg = configs.decode_fp8(seed=820, ctx=ctx)
+    out, lse = decode_cfg(cfg)
+    ro, rl = oracle.decode(cfg)
+    parity(out, lse, ro, rl, "fp8 split boundaries")
+    sink = synth.normal_f32(synth.stream_seed(821, 9), (64,))
+    cfg.layer = configs.Layer("swa", 4, 1e7, 1000, sink)
+    out, lse = decode_cfg(cfg)
+    ro, rl = oracle.decode(cfg)
+    parity(out, lse, ro, rl, "fp8 paged, window 1000 with sink")
+
+
+def test_decode_fp8_config3_scale():
+    """64 sequences, contexts U[4096, 65536] over an E4M3 paged cache, checked on 8 sequences."""
+    import torch
+    cfg = configs.decode_fp8()
+    out, lse = decode_cfg(cfg)
+    seqs = np.array(sorted(set([0, 63] + list(synth.permutation(79, 64)[:6]))))
+    ro, rl = oracle.decode(cfg, seqs=seqs)
+    idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "fp8 config-3 scale, sampled sequences")
 
 
 @pytest.fixture(scope="module")

@@ -403,3 +403,43 @@ def test_kv_append_oracle():
     for t in range(5):
         for g in range(2):
             np.testing.assert_array_equal(ko[t, g], oracle.rope(widen(k[t, g]), pos[t], 1e7, 64))
+
+
+# ----------------------------------------------------------------------------- E4M3 KV caches
+
+def test_e4m3_decoding_matches_torch_and_the_format_definition():
+    """The oracle's E4M3 decoding against torch.float8_e4m3fn (an independent library
+    implementation) for all 256 bytes, and against the format's fixed points."""
+    codes = np.arange(256)
+    mine = oracle.e4m3_to_double(codes)
+    ref = torch.from_numpy(codes.astype(np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert set(np.flatnonzero(nan)) == {0x7F, 0xFF}
+    np.testing.assert_array_equal(np.isnan(mine), nan)
+    np.testing.assert_array_equal(mine[~nan], ref[~nan])
+    fixed = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x39: 1.125,
+             0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    for c, v in fixed.items():
+        assert mine[c] == v, hex(c)
+
+
+def test_fp8_cache_equals_the_same_values_in_the_bf16_cache():
+    """Decoding over an E4M3 cache with power-of-two scales is the decoding over a cache in
+    the bf16 format that holds the dequantised values exactly (fp16 for the rotated dims):
+    the two paths of the oracle must agree bit for bit."""
+    from workloads import configs
+    cfg = configs.decode_fp8(seed=41, B=3, ctx_range=(200, 700))
+    cfg.k_dequant = np.array([0.5, 2.0, 1.0, 0.25], np.float32)
+    cfg.v_dequant = np.array([4.0, 1.0, 0.5, 2.0], np.float32)
+    ro, rl = oracle.decode(cfg)
+    kv = oracle.e4m3_to_double(cfg.k_cache) * cfg.k_dequant[None, None, :, None]
+    vv = oracle.e4m3_to_double(cfg.v_cache) * cfg.v_dequant[None, None, :, None]
+    kc = np.empty(kv.shape, np.uint16)
+    kc[..., :64] = synth.f64_to_f16_bits(kv[..., :64])
+    kc[..., 64:] = synth.f64_to_bf16_bits(kv[..., 64:])
+    assert np.array_equal(oracle.e4m3_to_double(cfg.k_cache)[..., 64:] * cfg.k_dequant[None, None, :, None],
+                          widen(kc[..., 64:]))
+    plain = configs.Decode(cfg.layer, cfg.q, cfg.ctx, kc, synth.f64_to_bf16_bits(vv), block_table=cfg.block_table)
+    po, pl = oracle.decode(plain)
+    np.testing.assert_array_equal(ro, po)
+    np.testing.assert_array_equal(rl, pl)

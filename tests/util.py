@@ -16,6 +16,11 @@ def dev_bf16(a: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+def dev_u8(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
 def dev_i32(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.int32))).cuda()
@@ -65,10 +70,14 @@ def decode_cfg(cfg, **kw):
                      num_pages=cfg.k_cache.shape[0])
     else:
         extra = dict(cache_kind=M.MIMO_CACHE_RING)
+    if cfg.cache_dtype == M.MIMO_DTYPE_FP8_E4M3:
+        kc, vc = dev_u8(cfg.k_cache), dev_u8(cfg.v_cache)
+        extra.update(cache_dtype=cfg.cache_dtype, k_dequant=dev_f32(cfg.k_dequant), v_dequant=dev_f32(cfg.v_dequant))
+    else:
+        kc, vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
     return M.mimo_attn_decode(dev_bf16(cfg.q), dev_i32(cfg.ctx), max_seq_len=int(cfg.ctx.max()),
                               num_kv_heads=L.num_kv_heads, rope_base=L.rope_base, window=L.window,
-                              k_cache=dev_bf16(cfg.k_cache), v_cache=dev_bf16(cfg.v_cache), sink=dev_f32(L.sink),
-                              **extra, **kw)
+                              k_cache=kc, v_cache=vc, sink=dev_f32(L.sink), **extra, **kw)
 
 
 def chunked_cfg(cfg):

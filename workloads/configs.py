@@ -78,6 +78,25 @@ def bf16_normal(seed: int, tag: int, shape) -> np.ndarray:
     return _normal_bf16_parallel(synth.stream_seed(seed, tag), shape)
 
 
+def fp8_codes(seed: int, tag: int, shape) -> np.ndarray:
+    """Synthetic E4M3 cache bytes: sign and 3 mantissa bits uniform, exponent field uniform
+    in 4..8, i.e. magnitudes (1 + m/8) * 2^(e-7) in [0.125, 3.75]."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+    step = 1 << 24
+    key = synth.stream_seed(seed, tag)
+
+    def work(lo):
+        hi = min(n, lo + step)
+        u = synth.u64(synth.stream_seed(key, lo // step), hi - lo)
+        e = (np.uint64(4) + (u >> np.uint64(4)) % np.uint64(5)).astype(np.uint8)
+        out[lo:hi] = ((u & np.uint64(1)).astype(np.uint8) << 7) | (e << 3) | ((u >> np.uint64(1)) & np.uint64(7)).astype(np.uint8)
+
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, range(0, n, step)))
+    return out.reshape(shape)
+
+
 def cached_keys(seed: int, tag: int, shape) -> np.ndarray:
     """~N(0,1) key rows [..., 192] in the cache format: dims 0..63 (the rotated part)
     as IEEE fp16 bit patterns, dims 64..191 as bf16 bit patterns."""
@@ -141,6 +160,9 @@ class Decode:
     v_cache: np.ndarray
     block_table: np.ndarray | None = None   # int32 [B, max_pages] (paged only)
     name: str = ""
+    cache_dtype: int = 0                     # 0: bf16 rows (fp16 rotated dims); 1: E4M3 bytes
+    k_dequant: np.ndarray | None = None      # fp32 [Hkv] dequantisation scales (E4M3 caches)
+    v_dequant: np.ndarray | None = None
 
     @property
     def paged(self) -> bool:
@@ -267,6 +289,27 @@ def verify(seed: int = BASE_SEED + 5, B: int = 64, q_len: int = 4, ctx_range=(40
                   bf16_normal(seed, 23, (n, 8, DV)), cu, start, cached_keys(seed, 25, (B, RING, 8, DQK)),
                   bf16_normal(seed, 26, (B, RING, 8, DV)), name=f"swa_verify_b{B}_q{q_len}")
     return glb, swa
+
+
+def decode_fp8(seed: int = BASE_SEED + 6, B: int = 64, ctx_range=(4096, 65536), ring: bool = False,
+               ctx: np.ndarray | None = None) -> Decode:
+    """Decode step over an E4M3 KV cache with per-KV-head scales: the global layer over a
+    paged cache (contexts uniform in ctx_range, or `ctx`), or the SWA layer over the ring."""
+    if ctx is None:
+        ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
+    B = len(ctx)
+    if ring:
+        L = swa_layer(synth.normal_f32(synth.stream_seed(seed, 4), (HQ,)))
+        h, shape_k, shape_v, bt = 8, (B, RING, 8, DQK), (B, RING, 8, DV), None
+    else:
+        L = global_layer()
+        bt, pool = paged_layout(seed, 10, ctx)
+        h, shape_k, shape_v = 4, (pool, PAGE, 4, DQK), (pool, PAGE, 4, DV)
+    ks = (0.5 + synth.uniform01(synth.stream_seed(seed, 7), h)).astype(np.float32)
+    vs = (0.5 + synth.uniform01(synth.stream_seed(seed, 8), h)).astype(np.float32)
+    return Decode(L, bf16_normal(seed, 1, (B, HQ, DQK)), ctx, fp8_codes(seed, 2, shape_k), fp8_codes(seed, 3, shape_v),
+                  block_table=bt, name=f"{'swa' if ring else 'global'}_decode_b{B}_fp8", cache_dtype=1,
+                  k_dequant=ks, v_dequant=vs)
 
 
 def sample_rows(seed: int, n_total: int, n_sample: int, always=()) -> np.ndarray:
