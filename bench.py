@@ -39,9 +39,10 @@ FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) p
 # The step's dominant kernel (about 97% of the step's device time in the ncu launch list).
 DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
-# workload, from the ncu capture summarised in profiles/; absent (null in the line) until the
-# current kernel has been captured.
-TRAFFIC_BYTES = {}
+# workload, from the ncu capture summarised in profiles/prefill_swa_kernel_2x4096_full.md
+# (kernel at commit 4bd734f): 249.66 MB read + 104.12 MB written for 2 x 4096 tokens, scaled
+# by tokens to the 40696-token workload.  Removed whenever the kernel changes.
+TRAFFIC_BYTES = {"prefill_swa_kernel": int((249.656832e6 + 104.123392e6) * 40696 / 8192)}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
