@@ -73,8 +73,9 @@ struct Layout {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffSeq = kOffMisc + 16;                       // int [6][kMaxSeqs + 1]
   static constexpr int kOffSink = kOffSeq + 6 * (kMaxSeqs + 1) * 4;   // float [64], log2 units
-  static constexpr int kOffCS = kOffSink + 64 * 4;                    // float2 [R][32] cos/sin of a tile
+  static constexpr int kOffCS = (kOffSink + 64 * 4 + 15) / 16 * 16;  // float2 [R][32] cos/sin of a tile
   static constexpr int kBytes = kOffCS + C::R * 32 * 8;
+  static_assert(kOffBar % 8 == 0 && kOffSeq % 4 == 0 && kOffCS % 16 == 0, "mbarrier / table / vector alignment");
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -625,6 +626,7 @@ struct SwaLayout {
   static constexpr int kBytes = kOffStage + 8 * kStageBytes;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(kOffBar % 8 == 0 && kOffSeq % 4 == 0 && kOffStage % 16 == 0, "mbarrier / table / vector alignment");
   static_assert(kOffCS % 128 == 0 && kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
                 "TMA destinations: 1024-byte aligned for 128-byte swizzle, 128-byte otherwise");
 };
