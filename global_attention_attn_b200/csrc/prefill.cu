@@ -503,7 +503,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           }
         }
         const float mt_l2 = mx * c_log2;
-        if (j > 0 && !(ok = wait_w(pv_done, (jj - 1) & 1))) break;
         const float m_new = fmaxf(m_run, mt_l2);
         float alpha = 1.f;
         const bool resc = m_new > m_run + 8.f;
@@ -511,7 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           alpha = ex2(m_run - m_new);
           m_run = m_new;
         }
+        // Only a rescale of O needs PV(j-1) to have landed: P(j) goes to the other S buffer,
+        // whose previous P was read by PV(j-2), which completed before QK(j) (in-order MMAs).
         if (__any_sync(0xffffffffu, resc && j > 0)) {
+          if (!(ok = wait_w(pv_done, (jj - 1) & 1))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 128; c += 32) {
