@@ -412,7 +412,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--main-only", action="store_true", help="skip the per-config details and the CPU baseline")
-    ap.add_argument("--profile", choices=["swa", "global", "decode", "decode_fp8"],
+    ap.add_argument("--profile", choices=["swa", "global", "decode", "decode_fp8", "swa_chunk"],
                     help="run only a small case of one kernel (inputs > L2, < 1 GB on the device) for ncu captures")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
@@ -597,6 +597,8 @@ def profile_case(name):
         return Prefill(configs.config2(S=4096))
     if name == "decode_fp8":
         return Decode(configs.decode_fp8(B=16))
+    if name == "swa_chunk":
+        return Chunked(configs.config4(n_sample=8)[1])
     sw, gl = configs.config3(B=16)
     return Decode(gl)
 

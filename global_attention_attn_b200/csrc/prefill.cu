@@ -554,7 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int qs = (mt + 1) % NQ;
         if (!(ok = wait_w(q_full(qs), ((mt + 1) / NQ) & 1) && rotate_q(Tn, qs))) break;
       }
-      // ---- epilogue
+      // ---- epilogue: O is final once the PVs of this tile's last two key tiles landed.
+      // The softmax waits for a PV only when it rescales O, so both may still be pending
+      // here, and a single parity wait could be met by the phase before them: wait in order.
+      if (nkv >= 2 && !(ok = wait_w(pv_done, (jj - 2) & 1))) break;
       if (!(ok = wait_w(pv_done, (jj - 1) & 1))) break;
       tc_fence_after();
       const float sc = p.v_scale / l_run;
