@@ -110,7 +110,6 @@ struct RopeKParams {
   int total_q;
   const int32_t* cu_q;
   float2* cs_q;    // [total_q, 32]
-  int key_blocks;  // blocks of the launch that work on keys; the rest fill cs_q
   RopeFreqs rope;
   unsigned* status;
 };

@@ -1122,100 +1122,193 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
 }
 
 // ---------------------------------------------------------------- key pre-pass
-// contig: 4 lanes per (row, kv head) write rotated dims 0..63 (fp16) into ws_k.
-// ext: one warp per (ext row, kv head) writes the full rotated key (dims 0..63
-//      fp16, 64..191 bf16) and the value: halo rows copied from the ring (which
-//      stores the same format), new rows rotated from k / v.
-__global__ void __launch_bounds__(256) rope_k_kernel(const RopeKParams p) {
-  if (int(blockIdx.x) >= p.key_blocks) {
-    // (cos, sin) of the 32 rotary frequencies at each query row's position: one warp per row
-    const long row = (long(blockIdx.x - p.key_blocks) * blockDim.x + threadIdx.x) >> 5;
-    const int j = threadIdx.x & 31;
-    if (row >= p.total_q) return;
-    int lo = 0, hi = p.num_seqs;  // sequence of the row
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.cu_q[mid] <= row) lo = mid; else hi = mid;
-    }
-    const int qlen = p.cu_q[lo + 1] - p.cu_q[lo];
-    const int ctx = (p.cache_lens ? p.cache_lens[lo] : 0) + (p.cu_k[lo + 1] - p.cu_k[lo]);
-    const int pos = ctx - qlen + int(row - p.cu_q[lo]);
-    float c, sn;
-    rope_cos_sin(pos, p.rope.inv_freq[j], &c, &sn);
-    p.cs_q[row * kHalf + j] = make_float2(c, sn);
-    return;
+// Position of query row `row` (its sequence found by bisection of cu_q): the queries of a
+// sequence are the last q_len of its ctx = cached + new keys.
+__device__ __forceinline__ int query_position(const RopeKParams& p, long row) {
+  int lo = 0, hi = p.num_seqs;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.cu_q[mid] <= row) lo = mid; else hi = mid;
   }
+  const int qlen = p.cu_q[lo + 1] - p.cu_q[lo];
+  const int ctx = (p.cache_lens ? p.cache_lens[lo] : 0) + (p.cu_k[lo + 1] - p.cu_k[lo]);
+  return ctx - qlen + int(row - p.cu_q[lo]);
+}
+
+// contig: one thread per (row, u = frequencies 8u..8u+7).  For key rows it writes the
+// rotated dims 0..63 (fp16) of all HKV heads into ws_k: the heads share the row's
+// position, so the 8 (cos, sin) pairs are computed once, and the loads of every head are
+// issued before the trig so that their latency overlaps it.  For query rows (when cs_q is
+// set) it writes the same 8 pairs at the query's position, reusing the key's pairs when
+// the two positions agree (prefill without a cache).
+template <int HKV>
+__global__ void __launch_bounds__(256, 2) rope_k_contig_kernel(const RopeKParams p) {
   const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (p.mode == kModeContig) {
-    const long item = gt >> 2;
-    const int u = int(gt & 3);
-    if (item >= long(p.total_k) * p.hkv) return;
-    const int row = int(item / p.hkv), g = int(item % p.hkv);
+  const long row = gt >> 2;
+  const int u = int(gt & 3);
+  const bool key_row = row < p.total_k;
+  const bool q_row = p.cs_q && row < p.total_q;
+  if (!key_row && !q_row) return;
+  uint4 a[HKV], b[HKV];
+  int pos_k = 0;
+  float2 cs[8];
+  if (key_row) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.k + row * HKV * kDqk) + u;
+#pragma unroll
+    for (int g = 0; g < HKV; ++g) {
+      a[g] = __ldg(src + g * (kDqk / 8));
+      b[g] = __ldg(src + g * (kDqk / 8) + 4);
+    }
     int lo = 0, hi = p.num_seqs;  // find s with cu_k[s] <= row < cu_k[s+1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (p.cu_k[mid] <= row) lo = mid; else hi = mid;
     }
-    const int pos = (p.cache_lens ? p.cache_lens[lo] : 0) + (row - p.cu_k[lo]);
-    const uint4* src = reinterpret_cast<const uint4*>(p.k + (long(row) * p.hkv + g) * kDqk);
-    uint4 a = __ldg(src + u), b = __ldg(src + u + 4);
-    rope_chunk_pair(a, b, u, pos, p.rope);
-    uint4* dst = reinterpret_cast<uint4*>(p.ws_k + (long(row) * p.hkv + g) * kRope);
-    dst[u] = a;
-    dst[u + 4] = b;
-    return;
-  }
-  const long wid = gt >> 5;
-  const int lane = int(gt & 31);
-  const long rows = long(p.total_k) + 128L * p.num_seqs;
-  if (wid >= rows * p.hkv) return;
-  const int e = int(wid / p.hkv), g = int(wid % p.hkv);
-  int lo = 0, hi = p.num_seqs;  // ext start of s: cu_k[s] + 128 s
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (p.cu_k[mid] + 128 * mid <= e) lo = mid; else hi = mid;
-  }
-  const int s = lo, i = e - (p.cu_k[s] + 128 * s);
-  const int clen = p.cache_lens ? p.cache_lens[s] : 0;
-  uint4* kd = reinterpret_cast<uint4*>(p.ws_k + (long(e) * p.hkv + g) * kDqk);
-  uint4* vd = reinterpret_cast<uint4*>(p.ws_v + (long(e) * p.hkv + g) * kDv);
-  if (i < 128) {
-    const int pos = clen - 128 + i;
-    if (pos < 0) {
-      if (lane < 24) kd[lane] = make_uint4(0, 0, 0, 0);
-      if (lane < 16) vd[lane] = make_uint4(0, 0, 0, 0);
-      return;
+    pos_k = (p.cache_lens ? p.cache_lens[lo] : 0) + int(row - p.cu_k[lo]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rope_cos_sin(pos_k, p.rope.inv_freq[8 * u + i], &cs[i].x, &cs[i].y);
+    uint4* dst = reinterpret_cast<uint4*>(p.ws_k + row * HKV * kRope) + u;
+#pragma unroll
+    for (int g = 0; g < HKV; ++g) {
+      rope_chunk_pair_cs(a[g], b[g], cs);
+      dst[g * (kRope / 8)] = a[g];
+      dst[g * (kRope / 8) + 4] = b[g];
     }
-    const long entry = long(s) * kPage + (pos % kPage);
-    const uint4* ks = reinterpret_cast<const uint4*>(p.ring_k + (entry * p.hkv + g) * kDqk);
-    const uint4* vs = reinterpret_cast<const uint4*>(p.ring_v + (entry * p.hkv + g) * kDv);
-    if (lane < 24) kd[lane] = __ldg(ks + lane);
-    if (lane < 16) vd[lane] = __ldg(vs + lane);
-    return;
   }
-  const int row = p.cu_k[s] + (i - 128);
-  const int pos = clen + (i - 128);
-  const uint4* ks = reinterpret_cast<const uint4*>(p.k + (long(row) * p.hkv + g) * kDqk);
-  if (lane < 4) {
-    uint4 a = __ldg(ks + lane), b = __ldg(ks + lane + 4);
-    rope_chunk_pair(a, b, lane, pos, p.rope);
-    kd[lane] = a;
-    kd[lane + 4] = b;
-  } else if (lane >= 8 && lane < 24) {
-    kd[lane] = __ldg(ks + lane);
+  if (q_row) {
+    const int pos_q = query_position(p, row);
+    if (!key_row || pos_q != pos_k) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rope_cos_sin(pos_q, p.rope.inv_freq[8 * u + i], &cs[i].x, &cs[i].y);
+    }
+    float4* d = reinterpret_cast<float4*>(p.cs_q + row * kHalf + 8 * u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_float4(cs[2 * i].x, cs[2 * i].y, cs[2 * i + 1].x, cs[2 * i + 1].y);
   }
-  if (lane < 16) vd[lane] = __ldg(reinterpret_cast<const uint4*>(p.v + (long(row) * p.hkv + g) * kDv) + lane);
+}
+
+// ext: one warp per row e of [128-slot ring halo | new keys] of each sequence.  It writes
+// the whole key of all HKV heads (dims 0..63 rotated fp16, 64..191 bf16) and the value:
+// halo rows are copied from the ring (which holds that format; zeros before the sequence
+// start), new rows are rotated from k / v.  Lane j computes frequency j's (cos, sin)
+// once; lane l rotates chunk pair (head l / 4, u = l % 4) with the pairs of frequencies
+// 8u..8u+7 taken from the lanes that hold them.  The same warp also fills query row e's
+// cos/sin row when cs_q is set.
+template <int HKV>
+__global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
+  static_assert(HKV * 4 <= 32, "one rotated chunk pair per lane");
+  constexpr int kKRow = HKV * kDqk / 8;  // uint4 of one position's keys (all heads)
+  constexpr int kVRow = HKV * kDv / 8;
+  const long wid = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long rows = long(p.total_k) + 128L * p.num_seqs;
+  const bool key_row = wid < rows;
+  const bool q_row = p.cs_q && wid < p.total_q;
+  if (!key_row && !q_row) return;
+  int pos_k = 0;
+  bool have_cs = false;  // c_j, s_j hold frequency `lane` at pos_k (warp-uniform)
+  float c_j = 0.f, s_j = 0.f;
+  if (key_row) {
+    const int e = int(wid);
+    int lo = 0, hi = p.num_seqs;  // ext start of s: cu_k[s] + 128 s
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.cu_k[mid] + 128 * mid <= e) lo = mid; else hi = mid;
+    }
+    const int s = lo, i = e - (p.cu_k[s] + 128 * s);
+    const int clen = p.cache_lens ? p.cache_lens[s] : 0;
+    uint4* kd = reinterpret_cast<uint4*>(p.ws_k + long(e) * HKV * kDqk);
+    uint4* vd = reinterpret_cast<uint4*>(p.ws_v + long(e) * HKV * kDv);
+    if (i < 128) {
+      const int pos = clen - 128 + i;
+      if (pos < 0) {
+        for (int t = lane; t < kKRow; t += 32) kd[t] = make_uint4(0, 0, 0, 0);
+        for (int t = lane; t < kVRow; t += 32) vd[t] = make_uint4(0, 0, 0, 0);
+      } else {
+        const long entry = long(s) * kPage + (pos % kPage);
+        const uint4* ks = reinterpret_cast<const uint4*>(p.ring_k + entry * HKV * kDqk);
+        const uint4* vs = reinterpret_cast<const uint4*>(p.ring_v + entry * HKV * kDv);
+        uint4 kr[(kKRow + 31) / 32], vr[(kVRow + 31) / 32];
+#pragma unroll
+        for (int t = 0; t < (kKRow + 31) / 32; ++t)
+          if (lane + 32 * t < kKRow) kr[t] = __ldg(ks + lane + 32 * t);
+#pragma unroll
+        for (int t = 0; t < (kVRow + 31) / 32; ++t)
+          if (lane + 32 * t < kVRow) vr[t] = __ldg(vs + lane + 32 * t);
+#pragma unroll
+        for (int t = 0; t < (kKRow + 31) / 32; ++t)
+          if (lane + 32 * t < kKRow) kd[lane + 32 * t] = kr[t];
+#pragma unroll
+        for (int t = 0; t < (kVRow + 31) / 32; ++t)
+          if (lane + 32 * t < kVRow) vd[lane + 32 * t] = vr[t];
+      }
+    } else {
+      const long row = p.cu_k[s] + (i - 128);
+      pos_k = clen + (i - 128);
+      const uint4* ks = reinterpret_cast<const uint4*>(p.k + row * HKV * kDqk);
+      const uint4* vs = reinterpret_cast<const uint4*>(p.v + row * HKV * kDv);
+      // rotated pair of this lane, the plain key chunks (dims 64..191) and the value
+      constexpr int kPlain = HKV * 16 / 32, kVal = kVRow / 32;
+      const int pg = lane >> 2, pu = lane & 3;
+      const bool has_pair = pg < HKV;
+      uint4 ra, rb, kp[kPlain], vv[kVal];
+      if (has_pair) {
+        ra = __ldg(ks + pg * (kDqk / 8) + pu);
+        rb = __ldg(ks + pg * (kDqk / 8) + pu + 4);
+      }
+#pragma unroll
+      for (int t = 0; t < kPlain; ++t) {
+        const int c = lane + 32 * t;
+        kp[t] = __ldg(ks + (c >> 4) * (kDqk / 8) + 8 + (c & 15));
+      }
+#pragma unroll
+      for (int t = 0; t < kVal; ++t) vv[t] = __ldg(vs + lane + 32 * t);
+      rope_cos_sin(pos_k, p.rope.inv_freq[lane], &c_j, &s_j);
+      have_cs = true;
+      float2 cs[8];
+#pragma unroll
+      for (int f = 0; f < 8; ++f) {
+        cs[f].x = __shfl_sync(0xffffffffu, c_j, 8 * pu + f);
+        cs[f].y = __shfl_sync(0xffffffffu, s_j, 8 * pu + f);
+      }
+      if (has_pair) {
+        rope_chunk_pair_cs(ra, rb, cs);
+        kd[pg * (kDqk / 8) + pu] = ra;
+        kd[pg * (kDqk / 8) + pu + 4] = rb;
+      }
+#pragma unroll
+      for (int t = 0; t < kPlain; ++t) {
+        const int c = lane + 32 * t;
+        kd[(c >> 4) * (kDqk / 8) + 8 + (c & 15)] = kp[t];
+      }
+#pragma unroll
+      for (int t = 0; t < kVal; ++t) vd[lane + 32 * t] = vv[t];
+    }
+  }
+  if (q_row) {
+    const int pos_q = query_position(p, wid);
+    if (!have_cs || pos_q != pos_k) rope_cos_sin(pos_q, p.rope.inv_freq[lane], &c_j, &s_j);
+    p.cs_q[wid * kHalf + lane] = make_float2(c_j, s_j);
+  }
 }
 
 cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s) {
-  long threads;
-  if (p.mode == kModeContig) threads = long(p.total_k) * p.hkv * 4;
-  else threads = (long(p.total_k) + 128L * p.num_seqs) * p.hkv * 32;
-  RopeKParams q = p;
-  q.key_blocks = int((threads + 255) / 256);
-  const long cs_blocks = q.cs_q ? (long(q.total_q) * 32 + 255) / 256 : 0;
-  if (q.key_blocks + cs_blocks == 0) return cudaSuccess;
-  rope_k_kernel<<<unsigned(q.key_blocks + cs_blocks), 256, 0, s>>>(q);
+  if (p.hkv != 4 && p.hkv != 8) return cudaErrorInvalidValue;
+  const long qrows = p.cs_q ? long(p.total_q) : 0;
+  if (p.mode == kModeContig) {
+    const long rows = long(p.total_k) > qrows ? long(p.total_k) : qrows;
+    const long blocks = (rows * 4 + 255) / 256;
+    if (blocks == 0) return cudaSuccess;
+    if (p.hkv == 8) rope_k_contig_kernel<8><<<unsigned(blocks), 256, 0, s>>>(p);
+    else rope_k_contig_kernel<4><<<unsigned(blocks), 256, 0, s>>>(p);
+  } else {
+    const long ext = long(p.total_k) + 128L * p.num_seqs;
+    const long rows = ext > qrows ? ext : qrows;
+    const long blocks = (rows * 32 + 255) / 256;
+    if (blocks == 0) return cudaSuccess;
+    if (p.hkv == 8) rope_k_ext_kernel<8><<<unsigned(blocks), 256, 0, s>>>(p);
+    else rope_k_ext_kernel<4><<<unsigned(blocks), 256, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -296,9 +296,16 @@ def test_prefill_swa_small_window():
     check_prefill(make_prefill([300], 8, 1e4, 5, True, 303), what="swa window 5")
 
 
-def test_prefill_swa_fewer_queries_than_keys():
-    # bottom-right alignment: 40 queries at the end of 300 keys
-    check_prefill(make_prefill([40], 8, 1e4, 128, True, 304, klens=[300]), what="swa q<k")
+@pytest.mark.parametrize("lens,klens", [([40], [300]), ([40, 17, 130, 1], [300, 17, 500, 64])],
+                         ids=["one", "mixed"])
+def test_prefill_swa_fewer_queries_than_keys(lens, klens):
+    # bottom-right alignment: each sequence's queries sit at the end of its keys, so the
+    # query cos/sin rows are at other positions than the key rows of the same index
+    check_prefill(make_prefill(lens, 8, 1e4, 128, True, 304, klens=klens), what="swa q<k")
+
+
+def test_prefill_global_fewer_queries_than_keys():
+    check_prefill(make_prefill([33, 200, 7], 4, 1e7, 0, False, 305, klens=[400, 200, 129]), what="global q<k")
 
 
 def test_prefill_config1_sampled():
