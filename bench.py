@@ -373,7 +373,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     import oracle
-    cfg = configs.config1()
+    cfg = configs.swa_varlen_prefill()
     cores = oracle.default_threads()
     total = int(cfg.cu_q[-1])
     # size each step's sample so that warmup + steps take about two minutes of CPU time
@@ -442,7 +442,7 @@ def main():
             pg.barrier()
 
     # ---------------- the timed workload: sliding-window varlen prefill
-    cfg = configs.config1()
+    cfg = configs.swa_varlen_prefill()
     flops, by = prefill_counts(cfg)
     step = Prefill(cfg)
     for _ in range(args.warmup):
@@ -515,7 +515,7 @@ def main():
         torch.cuda.empty_cache()
         per = {}
         flush = l2_flusher()
-        c0 = configs.config0()
+        c0 = configs.swa_prefill_s512()
         f0, b0 = prefill_counts(c0)
         w0 = Prefill(c0)
         for _ in range(3):
@@ -523,7 +523,7 @@ def main():
         t0 = event_time_ms(w0, 50, flush=flush) / 50
         per["swa_prefill_s512"] = _entry(f0, b0, t0, hbm, tf_burst, "L2 flushed before each call")
         del w0
-        c2 = configs.config2()
+        c2 = configs.global_causal_prefill()
         f2, b2 = prefill_counts(c2)
         w2 = Prefill(c2)
         for _ in range(3):
@@ -532,7 +532,7 @@ def main():
         per["global_prefill_s16384"] = _entry(f2, b2, t2, hbm, tf_sust, "inputs larger than L2")
         del w2, c2
         torch.cuda.empty_cache()
-        sw, gl = configs.config3()
+        sw, gl = configs.decode_batch()
         for name, c, fl in (("swa_decode_b64_ring128", sw, flush), ("global_decode_b64_paged128", gl, None)):
             fd, bd = decode_counts(c)
             w = Decode(c)
@@ -565,7 +565,7 @@ def main():
             del w
         del sw, gl, vg, vs
         torch.cuda.empty_cache()
-        g4, s4 = configs.config4()
+        g4, s4 = configs.chunked_prefill()
         for name, c in (("global_chunk_8192_on_120832", g4), ("swa_chunk_8192_on_120832", s4)):
             fc, bc = chunked_counts(c)
             w = Chunked(c)
@@ -594,12 +594,12 @@ def profile_case(name):
         return Prefill(configs.Prefill(L, configs.bf16_normal(5, 1, (T, 64, 192)), configs.bf16_normal(5, 2, (T, 8, 192)),
                                        configs.bf16_normal(5, 3, (T, 8, 128)), cu, cu.copy(), name="swa_prefill_2x4096"))
     if name == "global":
-        return Prefill(configs.config2(S=4096))
+        return Prefill(configs.global_causal_prefill(S=4096))
     if name == "decode_fp8":
         return Decode(configs.decode_fp8(B=16))
     if name == "swa_chunk":
-        return Chunked(configs.config4(n_sample=8)[1])
-    sw, gl = configs.config3(B=16)
+        return Chunked(configs.chunked_prefill(n_sample=8)[1])
+    sw, gl = configs.decode_batch(B=16)
     return Decode(gl)
 
 

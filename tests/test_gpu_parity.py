@@ -150,7 +150,7 @@ def test_kv_append_fp8(kind):
 
 @pytest.mark.parametrize("ctx_range", [(1, 127), (100, 3000), (4096, 9000)])
 def test_decode_small(ctx_range):
-    sw, gl = configs.config3(seed=100 + ctx_range[0], B=8, ctx_range=ctx_range)
+    sw, gl = configs.decode_batch(seed=100 + ctx_range[0], B=8, ctx_range=ctx_range)
     for cfg in (sw, gl):
         out, lse = decode_cfg(cfg)
         ro, rl = oracle.decode(cfg)
@@ -160,7 +160,7 @@ def test_decode_small(ctx_range):
 def test_decode_split_boundaries():
     # contexts on both sides of the 512-key split length and of one page
     import global_attention_attn_b200 as M
-    sw, gl = configs.config3(seed=321, B=8, ctx_range=(1, 2))
+    sw, gl = configs.decode_batch(seed=321, B=8, ctx_range=(1, 2))
     ctx = np.array([1, 127, 128, 129, 511, 512, 513, 1025], np.int32)
     bt, pool = configs.paged_layout(5, 1, ctx)
     gl = configs.Decode(gl.layer, gl.q, ctx, configs.cached_keys(5, 2, (pool, 128, 4, 192)),
@@ -232,7 +232,7 @@ def test_decode_fp8_split_boundaries_and_window():
     parity(out, lse, ro, rl, "fp8 paged, window 1000 with sink")
 
 
-def test_decode_fp8_config3_scale():
+def test_decode_fp8_b64_full_scale():
     """64 sequences, contexts U[4096, 65536] over an E4M3 paged cache, checked on 8 sequences."""
     import torch
     cfg = configs.decode_fp8()
@@ -244,31 +244,31 @@ def test_decode_fp8_config3_scale():
 
 
 @pytest.fixture(scope="module")
-def cfg3():
-    return configs.config3()
+def dec64():
+    return configs.decode_batch()
 
 
-def test_decode_config3_swa_ring(cfg3):
-    sw, _ = cfg3
+def test_decode_b64_swa_ring(dec64):
+    sw, _ = dec64
     out, lse = decode_cfg(sw)
     ro, rl = oracle.decode(sw)
-    parity(out, lse, ro, rl, "config 3 swa ring, all 64 sequences")
+    parity(out, lse, ro, rl, "decode b64 swa ring, all 64 sequences")
 
 
-def test_decode_config3_global_paged(cfg3):
-    _, gl = cfg3
+def test_decode_b64_global_paged(dec64):
+    _, gl = dec64
     out, lse = decode_cfg(gl)
     seqs = np.array(sorted(set([0, 63] + list(synth.permutation(77, 64)[:6]))))
     ro, rl = oracle.decode(gl, seqs=seqs)
     import torch
     idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "config 3 global paged, sampled sequences")
+    parity(out[idx], lse[idx], ro, rl, "decode b64 global paged, sampled sequences")
 
 
 # ----------------------------------------------------------------------------- prefill: sliding window
 
-def test_prefill_config0():
-    check_prefill(configs.config0(), what="config 0")
+def test_prefill_swa_s512():
+    check_prefill(configs.swa_prefill_s512(), what="swa prefill s512")
 
 
 @pytest.mark.parametrize("lens", [[1], [16], [127, 128, 129], [1, 15, 16, 17, 31, 300], [1000]])
@@ -308,8 +308,8 @@ def test_prefill_global_fewer_queries_than_keys():
     check_prefill(make_prefill([33, 200, 7], 4, 1e7, 0, False, 305, klens=[400, 200, 129]), what="global q<k")
 
 
-def test_prefill_config1_sampled():
-    cfg = configs.config1()
+def test_prefill_swa_varlen_sampled():
+    cfg = configs.swa_varlen_prefill()
     cu = cfg.cu_q
     always = set()
     for s in range(cfg.num_seqs):
@@ -317,7 +317,7 @@ def test_prefill_config1_sampled():
             always.add(int(cu[s] + r))
         always.add(int(cu[s + 1] - 1))
     rows = configs.sample_rows(11, int(cu[-1]), 1024, always=sorted(always))
-    check_prefill(cfg, rows=rows, what="config 1 (sampled rows)")
+    check_prefill(cfg, rows=rows, what="swa varlen prefill (sampled rows)")
 
 
 # ----------------------------------------------------------------------------- prefill: global
@@ -331,34 +331,34 @@ def test_prefill_global_with_sink_and_wide_window():
     check_prefill(make_prefill([700], 4, 1e7, 300, True, 410), what="global window 300 + sink")
 
 
-def test_prefill_config2_sampled():
-    cfg = configs.config2()
+def test_prefill_global_s16384_sampled():
+    cfg = configs.global_causal_prefill()
     rows = configs.sample_rows(22, 16384, 96, always=(0, 1, 7, 8, 127, 128, 129, 8191, 16383))
-    check_prefill(cfg, rows=rows, what="config 2 (sampled rows)")
+    check_prefill(cfg, rows=rows, what="global prefill s16384 (sampled rows)")
 
 
 # ----------------------------------------------------------------------------- chunked prefill
 
 def test_chunked_small_unaligned():
-    glb, swa = configs.config4(seed=55, prefix=1000, chunk=300, n_sample=300)
+    glb, swa = configs.chunked_prefill(seed=55, prefix=1000, chunk=300, n_sample=300)
     for cfg in (glb, swa):
         out, lse = chunked_cfg(cfg)
         ro, rl = oracle.chunked(cfg, rows=np.arange(300))
         parity(out, lse, ro, rl, cfg.name)
 
 
-def test_chunked_config4():
-    glb, swa = configs.config4()
+def test_chunked_8192_on_120832():
+    glb, swa = configs.chunked_prefill()
     out, lse = chunked_cfg(swa)
     ro, rl = oracle.chunked(swa)
     import torch
     idx = torch.as_tensor(swa.sample_rows, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "config 4 swa chunk (1024 sampled rows)")
+    parity(out[idx], lse[idx], ro, rl, "swa chunk 8192 on 120832 (1024 sampled rows)")
     out, lse = chunked_cfg(glb)
     rows = configs.sample_rows(4, 8192, 48, always=(0, 126, 127, 128, 8191))
     ro, rl = oracle.chunked(glb, rows=rows)
     idx = torch.as_tensor(rows, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "config 4 global chunk (sampled rows)")
+    parity(out[idx], lse[idx], ro, rl, "global chunk 8192 on 120832 (sampled rows)")
 
 
 # ----------------------------------------------------------------------------- cross-path
@@ -377,11 +377,11 @@ def test_verify_draft_tokens(q_len):
         parity(out, lse, ro, rl, cfg.name)
 
 
-def test_verify_config3_scale(cfg3):
+def test_verify_b64_full_scale(dec64):
     """Verification at the decode workload's scale (64 sequences, contexts up to 64K) on the
     config-3 caches, checked on the rows of 4 sampled sequences."""
     import torch
-    _, gl = cfg3
+    _, gl = dec64
     glb, swa = configs.verify(B=64, q_len=4, decode=gl)
     seqs = np.array([0, 17, 42, 63])
     rows = (seqs[:, None] * 4 + np.arange(4)[None, :]).reshape(-1)

@@ -30,7 +30,7 @@ def test_noalloc_rejects_oversize_before_touching_the_device():
 
 
 def _case(seed, B, ctx_range):
-    _, gl = configs.config3(seed=seed, B=B, ctx_range=ctx_range)
+    _, gl = configs.decode_batch(seed=seed, B=B, ctx_range=ctx_range)
     L = gl.layer
     t = dict(q=dev_bf16(gl.q), ctx=dev_i32(gl.ctx), kc=dev_bf16(gl.k_cache), vc=dev_bf16(gl.v_cache),
              bt=dev_i32(gl.block_table), pool=gl.k_cache.shape[0], max_len=int(gl.ctx.max()), L=L)

@@ -190,7 +190,7 @@ class Chunked:
         return self.block_table is not None
 
 
-def config0(seed: int = BASE_SEED + 0) -> Prefill:
+def swa_prefill_s512(seed: int = BASE_SEED + 0) -> Prefill:
     """One SWA layer prefill, batch 1, seq 512."""
     S = 512
     L = swa_layer(synth.normal_f32(synth.stream_seed(seed, 4), (HQ,)))
@@ -199,13 +199,13 @@ def config0(seed: int = BASE_SEED + 0) -> Prefill:
                    np.array([0, S], np.int32), name="swa_prefill_s512")
 
 
-def config1_lengths(seed: int = BASE_SEED + 1) -> np.ndarray:
+def swa_varlen_lengths(seed: int = BASE_SEED + 1) -> np.ndarray:
     return synth.randint(synth.stream_seed(seed, 0), 8, 1024, 8192)
 
 
-def config1(seed: int = BASE_SEED + 1) -> Prefill:
+def swa_varlen_prefill(seed: int = BASE_SEED + 1) -> Prefill:
     """SWA layer varlen prefill: 8 sequences, lengths uniform in [1024, 8192]."""
-    lens = config1_lengths(seed)
+    lens = swa_varlen_lengths(seed)
     cu = np.zeros(9, np.int32)
     cu[1:] = np.cumsum(lens)
     T = int(cu[-1])
@@ -214,7 +214,7 @@ def config1(seed: int = BASE_SEED + 1) -> Prefill:
                    bf16_normal(seed, 3, (T, 8, DV)), cu, cu.copy(), name="swa_varlen_prefill_8x[1024,8192]")
 
 
-def config2(seed: int = BASE_SEED + 2, S: int = 16384) -> Prefill:
+def global_causal_prefill(seed: int = BASE_SEED + 2, S: int = 16384) -> Prefill:
     """Global layer causal prefill, batch 1, seq 16384, no sink."""
     L = global_layer()
     return Prefill(L, bf16_normal(seed, 1, (S, HQ, DQK)), bf16_normal(seed, 2, (S, 4, DQK)),
@@ -236,15 +236,15 @@ def paged_layout(seed: int, tag: int, ctx: np.ndarray, extra_pool: int = 0):
     return bt, total
 
 
-def config3_ctx(seed: int = BASE_SEED + 3, B: int = 64) -> np.ndarray:
+def decode_contexts(seed: int = BASE_SEED + 3, B: int = 64) -> np.ndarray:
     return synth.randint(synth.stream_seed(seed, 0), B, 4096, 65536).astype(np.int32)
 
 
-def config3(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536)) -> tuple[Decode, Decode]:
+def decode_batch(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536)) -> tuple[Decode, Decode]:
     """Decode step, batch B: the SWA layer over a 128-slot ring, the global layer over
     a paged cache (page 128) with contexts uniform in ctx_range."""
     if ctx_range == (4096, 65536) and B == 64:
-        ctx = config3_ctx(seed, B)
+        ctx = decode_contexts(seed, B)
     else:
         ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
     Ls = swa_layer(synth.normal_f32(synth.stream_seed(seed, 4), (HQ,)))
@@ -264,8 +264,8 @@ def verify(seed: int = BASE_SEED + 5, B: int = 64, q_len: int = 4, ctx_range=(40
     """Speculative-decoding verification: each sequence scores q_len draft tokens at
     positions [ctx - q_len, ctx) after a cached prefix of ctx - q_len tokens, for the
     global layer (paged cache, the drafts appended first) and the SWA layer (ring holding
-    the 128 prefix positions before the drafts).  With `decode` (a global-layer Decode of
-    config 3) its contexts, block tables and cache are reused; the drafts then overwrite
+    the 128 prefix positions before the drafts).  With `decode` (a global-layer Decode from
+    `decode_batch`) its contexts, block tables and cache are reused; the drafts then overwrite
     the cache rows of the last q_len positions when they are appended."""
     if decode is None:
         ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
@@ -319,7 +319,7 @@ def sample_rows(seed: int, n_total: int, n_sample: int, always=()) -> np.ndarray
     return np.array(sorted(rows), np.int32)
 
 
-def config4(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int = 8192,
+def chunked_prefill(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int = 8192,
             n_sample: int = 1024) -> tuple[Chunked, Chunked]:
     """Chunked prefill: `chunk` new tokens after a `prefix`-token cached prefix, for the
     global layer (paged cache) and the matching SWA layer (ring holding the prefix tail)."""
