@@ -37,7 +37,7 @@ V_SCALE = 0.707
 
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_prefill_workspace_size", "mimo_attn_decode",
            "mimo_attn_decode_workspace_size", "mimo_attn_decode_noalloc", "mimo_kv_append", "mimo_last_error",
-           "mimo_status_poll", "mimo_version")
+           "mimo_status_poll", "mimo_version", "mimo_window_from_left_right")
 DECODE_NOALLOC_MAX_BYTES = 16 << 20
 
 _P = C.c_void_p
@@ -109,6 +109,8 @@ def lib():
         L.mimo_status_poll.restype = C.c_int
         L.mimo_version.argtypes = []
         L.mimo_version.restype = C.c_char_p
+        L.mimo_window_from_left_right.argtypes = [C.c_int, C.c_int, C.POINTER(C.c_int)]
+        L.mimo_window_from_left_right.restype = C.c_int
         _lib = L
     return _lib
 
@@ -264,6 +266,14 @@ def mimo_kv_append(k_new, v_new, pos, seq_idx, *, rope_base: float, cache_kind: 
     a.num_pages = num_pages
     a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
     _check(lib().mimo_kv_append(C.byref(a), _stream(stream)))
+
+
+def mimo_window_from_left_right(left: int, right: int = 0) -> int:
+    """`window` (keys in total including the query) of the (left, right) window form:
+    (128, 0) -> 129, (127, 0) -> 128, (-1, 0) -> 0 (global)."""
+    w = C.c_int(0)
+    _check(lib().mimo_window_from_left_right(int(left), int(right), C.byref(w)))
+    return int(w.value)
 
 
 def status_poll() -> int:

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -155,6 +156,16 @@ extern "C" {
 const char* mimo_last_error(void) { return g_err; }
 
 const char* mimo_version(void) { return "libmimoattn 0.1 (sm_100a)"; }
+
+int mimo_window_from_left_right(int left, int right, int* window) {
+  const char* fn = "mimo_window_from_left_right";
+  if (!window) return fail(MIMO_ERR_INVALID_ARG, "%s: window is NULL", fn);
+  if (right != 0) return fail(MIMO_ERR_UNSUPPORTED, "%s: right = %d: the layers are causal (right must be 0)", fn, right);
+  if (left < -1 || left == INT_MAX)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: left must be -1 (unbounded) or in 0..INT_MAX-1 (got %d)", fn, left);
+  *window = left + 1;
+  return MIMO_OK;
+}
 
 size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_q, int total_k, int num_kv_heads, int cache_kind) {
   if (num_seqs < 0 || total_q < 0 || total_k < 0 || num_kv_heads <= 0) return 0;

@@ -74,6 +74,19 @@ typedef struct {
   const float* sink;   /* device fp32 [num_q_heads] sink logits, or NULL for no sink */
 } mimo_layer;
 
+/* The (left, right) form of the window, as the sliding-window layers are configured in
+ * the SGLang / miles stack (radixark miles docs "MiMo-V2.6-Flash", section 5.4 "Notable
+ * quirks", which sets the window as (128, 0) there against 128 keys in total in the HF
+ * and Megatron-Bridge code): a query at position p sees the keys at positions
+ * [p - left, p + right].  The layers are causal, so right must be 0; left = -1 means no
+ * left bound (a global layer).  Writes the equivalent `window` of mimo_layer (keys in
+ * total including the query: left + 1, or 0 for left = -1) to *window, so (128, 0)
+ * gives 129 and (127, 0) gives 128.
+ * Errors: MIMO_ERR_UNSUPPORTED for right != 0 (non-causal); MIMO_ERR_INVALID_ARG for
+ * left < -1, left + 1 overflowing an int, or window == NULL.  Host only: touches no
+ * device and launches nothing. */
+MIMO_API int mimo_window_from_left_right(int left, int right, int* window);
+
 #define MIMO_CACHE_NONE 0
 #define MIMO_CACHE_PAGED 1 /* [num_pages, 128, Hkv, D] pages of 128 positions, via block_table */
 #define MIMO_CACHE_RING 2  /* [num_seqs, 128, Hkv, D]: position p of sequence s in slot p % 128 */

@@ -182,3 +182,18 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.replace("Oracle", ""), f
+
+
+@pytest.mark.parametrize("left,window", [(128, 129), (127, 128), (0, 1), (-1, 0), (2**31 - 2, 2**31 - 1)])
+def test_window_from_left_right(left, window):
+    assert M.mimo_window_from_left_right(left, 0) == window
+
+
+@pytest.mark.parametrize("left,right,code", [(128, 1, "MIMO_ERR_UNSUPPORTED"), (127, -1, "MIMO_ERR_UNSUPPORTED"),
+                                             (-2, 0, "MIMO_ERR_INVALID_ARG"), (2**31 - 1, 0, "MIMO_ERR_INVALID_ARG")])
+def test_window_from_left_right_rejects(left, right, code):
+    with pytest.raises(M.MimoError) as e:
+        M.mimo_window_from_left_right(left, right)
+    assert e.value.code == getattr(M, code)
+    L = M.lib()
+    assert L.mimo_window_from_left_right(128, 0, None) == M.MIMO_ERR_INVALID_ARG

@@ -347,6 +347,23 @@ def test_chunked_small_unaligned():
         parity(out, lse, ro, rl, cfg.name)
 
 
+def test_chunked_swa_window_left_right_128_0():
+    """SGLang's (128, 0) window, i.e. 129 keys, on the ring-cache chunk path: the first rows
+    of the chunk reach back over all 128 halo positions of the ring."""
+    import dataclasses
+
+    import global_attention_attn_b200 as M
+    W = M.mimo_window_from_left_right(128, 0)
+    assert W == 129
+    _, swa = configs.chunked_prefill(seed=56, prefix=1000, chunk=300, n_sample=300)
+    L = swa.layer
+    swa = dataclasses.replace(swa, layer=configs.Layer(L.kind, L.num_kv_heads, L.rope_base, W, L.sink),
+                              name="swa_chunk_300_on_1000_window_129")
+    out, lse = chunked_cfg(swa)
+    ro, rl = oracle.chunked(swa, rows=np.arange(300))
+    parity(out, lse, ro, rl, swa.name)
+
+
 def test_chunked_8192_on_120832():
     glb, swa = configs.chunked_prefill()
     out, lse = chunked_cfg(swa)

@@ -225,27 +225,31 @@ def test_no_sink_equals_very_negative_sink():
 
 # ----------------------------------------------------------------------------- window / GQA invariants
 
-def test_window_sees_exactly_min_pos_plus_one_128_keys():
+@pytest.mark.parametrize("W", [128, 129])
+def test_window_sees_exactly_min_pos_plus_one_W_keys(W):
+    """W = 128 keys in total (HF / Megatron-Bridge) or 129 (SGLang's (128, 0) window,
+    radixark miles docs "MiMo-V2.6-Flash", section 5.4): the key at distance W - 1 is
+    visible, the one at distance W is not."""
     dims = dict(hq=2, hkv=1, dqk=8, dv=4, rope_dim=4)
     q, k, v, s = tiny(seed=12, S=300, sink=True, **dims)
-    base_out, _ = run(q, k, v, s, window=128, **dims)
+    base_out, _ = run(q, k, v, s, window=W, **dims)
     i = 250
-    for dist, changes in [(127, True), (128, False), (129, False), (0, True)]:
+    for dist, changes in [(W - 2, True), (W - 1, True), (W, False), (W + 1, False), (0, True)]:
         v2 = v.copy()
         v2[i - dist] = synth.f64_to_bf16_bits(widen(v2[i - dist]) + 3.0)
-        o, _ = run(q, k, v2, s, window=128, rows=[i], **dims)
+        o, _ = run(q, k, v2, s, window=W, rows=[i], **dims)
         assert (np.abs(o[0] - base_out[i]).max() > 1e-6) == changes, dist
     # a key after the query is never visible
     v2 = v.copy()
     v2[i + 1] = synth.f64_to_bf16_bits(widen(v2[i + 1]) + 3.0)
-    o, _ = run(q, k, v2, s, window=128, rows=[i], **dims)
+    o, _ = run(q, k, v2, s, window=W, rows=[i], **dims)
     assert np.abs(o[0] - base_out[i]).max() == 0
-    # early positions see pos + 1 keys: zero query -> lse = ln(pos + 1 + e^s)
+    # early positions see pos + 1 keys: zero query -> lse = ln(min(pos + 1, W) + e^s)
     q0 = q.copy()
     q0[:] = 0
-    _, l = run(q0, k, v, s, window=128, **dims)
-    for p in (0, 1, 126, 127, 128, 299):
-        assert abs(l[p, 0] - math.log(min(p + 1, 128) + math.exp(s[0]))) < 1e-12
+    _, l = run(q0, k, v, s, window=W, **dims)
+    for p in (0, 1, 126, 127, 128, 129, 299):
+        assert abs(l[p, 0] - math.log(min(p + 1, W) + math.exp(s[0]))) < 1e-12
 
 
 def test_window_at_least_sequence_is_global():
