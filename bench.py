@@ -453,12 +453,10 @@ def main():
         t_ms, k_ms = timed_steps_ms(step, args.steps)
     barrier()
     if pg:
-        t = torch.tensor([t_ms, k_ms], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        t_ms, k_ms = float(t[0].item()), float(t[1].item())
+        t_ms, k_ms = max_over_ranks([t_ms, k_ms], pg, "cuda")
     ms_step = t_ms / args.steps
     ms_kernel = k_ms / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, ms_step) / 1e12
     achieved = by / (ms_kernel * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "traffic": TRAFFIC_BYTES.get(DOMINANT),
@@ -493,10 +491,8 @@ def main():
     barrier()
     te = event_time_ms(e2e_step, ke) / ke
     if pg:
-        t = torch.tensor([te], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        te = float(t.item())
-    e2e = {"value": flops * world / (te * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        te, = max_over_ranks([te], pg, "cuda")
+    e2e = {"value": whole_job_rate(flops, world, te) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": te}
     del q_h, k_h, v_h, out_h, lse_h
 
@@ -581,6 +577,20 @@ def main():
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+def max_over_ranks(values, dist_mod, device):
+    """Elementwise maximum of per-rank times over all ranks (every rank receives it): a
+    replica run is as slow as its slowest GPU."""
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3)
 
 
 def profile_case(name):

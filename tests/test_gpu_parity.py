@@ -382,6 +382,46 @@ def test_chunked_8192_on_120832():
 
 # ----------------------------------------------------------------------------- speculative verification
 
+# ----------------------------------------------------------------------------- context parallelism
+
+@pytest.mark.parametrize("splits,window", [
+    ([[300, 200, 129], [140, 131, 500]], 128),       # every chunk fills the 128-slot ring alone
+    ([[50, 30, 200, 7, 250], [10, 300, 2, 128, 64]], 129),  # short chunks: rings relayed
+], ids=["independent", "relay_window_129"])
+def test_cp_halo_prefill_emulated_on_one_gpu(splits, window):
+    """Context-parallel sliding-window prefill with the ranks run one after another on one
+    GPU (no rank waits on another's kernel): each rank's outgoing ring is built by the
+    library's key append (on top of its incoming ring when its chunk is short), and its
+    chunk is prefilled over the incoming ring.  The rows of all ranks must equal the
+    oracle's prefill of the whole sequences."""
+    import torch
+
+    from global_attention_attn_b200 import cp
+    B, R = len(splits), len(splits[0])
+    cfg = make_prefill([sum(sp) for sp in splits], 8, 1e4, window, True, 306 + window)
+    cu = cfg.cu_q
+    q, k, v, sink = dev_bf16(cfg.q), dev_bf16(cfg.k), dev_bf16(cfg.v), dev_f32(cfg.layer.sink)
+    out = torch.empty((int(cu[-1]), 64, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((int(cu[-1]), 64), dtype=torch.float32, device="cuda")
+    recv_k, recv_v = cp.ring_buffers(B, 8, "cuda")
+    starts = [0] * B
+    for r in range(R):
+        n = [splits[s][r] for s in range(B)]
+        idx = torch.cat([torch.arange(int(cu[s]) + starts[s], int(cu[s]) + starts[s] + n[s]) for s in range(B)]).cuda()
+        ql, kl, vl = q[idx].contiguous(), k[idx].contiguous(), v[idx].contiguous()
+        send_k, send_v = cp.ring_buffers(B, 8, "cuda")
+        st = list(starts)
+        cp.outgoing_ring(recv_k, recv_v, send_k, send_v,
+                         lambda rk, rv: cp.fill_ring_tail(rk, rv, kl, vl, n, st, rope_base=1e4),
+                         cp.chunks_fill_ring(n))
+        o, l = cp.prefill_with_halo(ql, kl, vl, n, st, recv_k, recv_v, rope_base=1e4, window=window, sink=sink)
+        out[idx], lse[idx] = o, l
+        recv_k, recv_v = send_k, send_v
+        starts = [starts[s] + n[s] for s in range(B)]
+    ro, rl = oracle.prefill(cfg)
+    parity(out, lse, ro, rl, f"cp halo ({R} ranks emulated, window {window})")
+
+
 @pytest.mark.parametrize("q_len", [2, 5, 8])
 def test_verify_draft_tokens(q_len):
     """q_len draft tokens per sequence scored against the cache: the global layer appends them

@@ -1,0 +1,104 @@
+"""Multi-process host logic on CPU (gloo): the replica bench's max-over-ranks timing and the
+context-parallel halo exchange of the sliding-window layers.  No GPU: the exchange is
+checked on float32 rings whose slots carry position markers, written by a stand-in for
+the key-append kernel."""
+import datetime
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+RING = 128
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _init(rank: int, world: int, port: int):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+
+
+def _run(fn, world: int, *args):
+    mp.spawn(fn, args=(world, _free_port()) + args, nprocs=world, join=True)
+
+
+# ----------------------------------------------------------------------------- replica timing
+
+def _bench_worker(rank, world, port):
+    _init(rank, world, port)
+    try:
+        import bench
+        mx = bench.max_over_ranks([10.0 + rank, 5.0 - rank], dist, "cpu")
+        assert mx == [10.0 + world - 1, 5.0], mx
+        # value = units of all ranks over the slowest rank's time
+        assert bench.whole_job_rate(100.0, world, mx[0]) == pytest.approx(100.0 * world / (mx[0] * 1e-3))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_bench_times_are_the_max_over_ranks(world):
+    _run(_bench_worker, world)
+
+
+# ----------------------------------------------------------------------------- CP halo exchange
+
+def _marker(s: int, p: int) -> float:
+    return float(p + 1 + 1000 * s)
+
+
+def _cp_worker(rank, world, port, splits):
+    _init(rank, world, port)
+    try:
+        from global_attention_attn_b200 import cp
+        B, hkv = len(splits), 2
+        lens = [splits[s][rank] for s in range(B)]
+        starts = [sum(splits[s][:rank]) for s in range(B)]
+        recv_k, recv_v = cp.ring_buffers(B, hkv, "cpu", torch.float32)
+        send_k, send_v = cp.ring_buffers(B, hkv, "cpu", torch.float32)
+        fills = []
+
+        def fill(rk, rv):
+            # stand-in for fill_ring_tail: slot p % 128 of sequence s gets marker(s, p)
+            fills.append(1)
+            for s, (row0, pos0, m) in enumerate(cp.tail_ranges(lens, starts)):
+                assert row0 == sum(lens[:s]) + lens[s] - m and pos0 == starts[s] + lens[s] - m
+                for p in range(pos0, pos0 + m):
+                    rk[s, p % RING] = _marker(s, p)
+                    rv[s, p % RING] = -_marker(s, p)
+
+        cp.exchange_halo(send_k, send_v, recv_k, recv_v, fill, independent=cp.chunks_fill_ring(lens))
+        assert len(fills) == (1 if rank + 1 < world else 0)
+        # the received ring holds exactly the 128 positions before this rank's chunk
+        for s in range(B):
+            st = starts[s]
+            for slot in range(RING):
+                p = st - RING + (slot - (st - RING)) % RING
+                want = _marker(s, p) if p >= 0 else 0.0
+                assert torch.all(recv_k[s, slot] == want), (rank, s, slot, p, recv_k[s, slot, 0, 0].item())
+                assert torch.all(recv_v[s, slot] == -want), (rank, s, slot, p)
+        if rank == 0:
+            with pytest.raises(ValueError):
+                cp.swa_prefill_context_parallel(None, None, None, [5], [3], rope_base=1e4, window=128)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("splits", [
+    # every chunk >= 128 positions: one round, no rank waits for another's ring
+    [[200, 150], [300, 129]],
+    # short chunks: the rings are relayed and a ring carries positions of several chunks
+    [[50, 30, 200, 7], [300, 10, 5, 60]],
+    # mixed: rank 1 relays, ranks 0 and 2 fill their rings alone
+    [[130, 40, 500]],
+], ids=["independent", "relay", "mixed"])
+def test_cp_halo_exchange(splits):
+    _run(_cp_worker, len(splits[0]), splits)
