@@ -137,12 +137,19 @@ __device__ __forceinline__ void fill_seq_table(const PrefillParams& p, const Seq
 
 // Maps work item w to (sequence, tile, kv head) from the shared table; any
 // thread may call it.  Tiles of a sequence are ordered longest-first for
-// global attention.
+// global attention, in snake order over the rounds of the persistent grid.
 template <int KIND>
 __device__ __forceinline__ bool locate(const PrefillParams& p, const SeqTable& S, int w, TileInfo& T) {
   constexpr int R = Cfg<KIND>::R;
+  const int total = S.tile_start[p.num_seqs] * p.hkv;
+  if (w >= total) return false;
+  if (KIND == 1) {
+    // CTA i takes items i, i + grid, ...: reverse every other round of grid items, so the
+    // CTA that gets a round's longest tile gets the next round's shortest
+    const int G = int(gridDim.x), round = w / G, base = round * G;
+    if (round & 1) w = base + min(G, total - base) - 1 - (w - base);
+  }
   const int tt = w / p.hkv;
-  if (tt >= S.tile_start[p.num_seqs]) return false;
   int lo = 0, hi = p.num_seqs;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
