@@ -212,7 +212,7 @@ MIMO_API int mimo_attn_decode(const mimo_decode_args* args, void* stream);
 /*
  * Decode for callers that cannot allocate device memory.
  *
- * The paper has no counterpart: this is a deployment convenience.  Some callers
+ * No page describes this call: it is a deployment convenience.  Some callers
  * cannot call cudaMalloc at all: code running inside a CUDA graph capture
  * region, or runtimes whose only device memory is a fixed arena handed out by
  * someone else.  For them this entry point behaves exactly like
