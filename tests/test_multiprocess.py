@@ -102,3 +102,20 @@ def _cp_worker(rank, world, port, splits):
 ], ids=["independent", "relay", "mixed"])
 def test_cp_halo_exchange(splits):
     _run(_cp_worker, len(splits[0]), splits)
+
+
+# ----------------------------------------------------------------------------- CP host logic
+
+def test_cp_tail_ranges_and_modes():
+    from global_attention_attn_b200 import cp
+    # (first local row, first position, count) of the keys a later chunk's window reaches
+    assert cp.tail_ranges([300, 50, 128], [1000, 0, 7]) == [(172, 1172, 128), (300, 0, 50), (350, 7, 128)]
+    assert cp.chunks_fill_ring([128, 500]) and not cp.chunks_fill_ring([128, 127])
+
+
+def test_cp_rejects_windows_beyond_the_halo():
+    from global_attention_attn_b200 import cp
+    q = torch.zeros((4, 64, 192), dtype=torch.bfloat16)
+    for w in (0, 130):
+        with pytest.raises(ValueError):
+            cp.prefill_with_halo(q, None, None, [4], [0], None, None, rope_base=1e4, window=w)
