@@ -650,7 +650,7 @@ constexpr uint32_t kSwaColO = 72;     // O inside a region
 __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __grid_constant__ PrefillParams p) {
   using C = Cfg<0>;
   using Ly = SwaLayout;
-  constexpr int G = C::G, R = C::R, BN = C::BN;
+  constexpr int G = C::G, BN = C::BN;
   constexpr int CH = BN / 3;  // 48 columns per softmax chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

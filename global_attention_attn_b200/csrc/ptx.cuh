@@ -255,6 +255,8 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
 }
+// (the half an unpack does not return is "set but never used": diagnostic 550)
+#pragma nv_diag_suppress 550
 __device__ __forceinline__ float lo_f32(uint64_t v) {
   float lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
@@ -265,6 +267,7 @@ __device__ __forceinline__ float hi_f32(uint64_t v) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
   return hi;
 }
+#pragma nv_diag_default 550
 __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
