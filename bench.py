@@ -412,7 +412,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--main-only", action="store_true", help="skip the per-config details and the CPU baseline")
-    ap.add_argument("--profile", choices=["swa", "global", "decode", "decode_fp8", "swa_chunk"],
+    ap.add_argument("--profile", choices=["swa", "global", "decode", "decode_fp8", "decode_ring", "swa_chunk"],
                     help="run only a small case of one kernel (inputs > L2, < 1 GB on the device) for ncu captures")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
@@ -609,6 +609,10 @@ def profile_case(name):
         return Decode(configs.decode_fp8(B=16))
     if name == "swa_chunk":
         return Chunked(configs.chunked_prefill(n_sample=8)[1])
+    if name == "decode_ring":
+        # the 64-sequence sliding-window decode over its 128-slot rings (44.6 MB, below L2:
+        # the capture sees the kernel with warm caches)
+        return Decode(configs.decode_batch()[0])
     sw, gl = configs.decode_batch(B=16)
     return Decode(gl)
 
