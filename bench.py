@@ -610,8 +610,8 @@ def profile_case(name):
     if name == "swa_chunk":
         return Chunked(configs.chunked_prefill(n_sample=8)[1])
     if name == "decode_ring":
-        # the 64-sequence sliding-window decode over its 128-slot rings (44.6 MB, below L2:
-        # the capture sees the kernel with warm caches)
+        # the 64-sequence sliding-window decode over its 128-slot rings (44.6 MB, below L2;
+        # ncu's default cache control flushes the caches before each captured pass)
         return Decode(configs.decode_batch()[0])
     sw, gl = configs.decode_batch(B=16)
     return Decode(gl)
