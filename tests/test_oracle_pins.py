@@ -447,3 +447,25 @@ def test_fp8_cache_equals_the_same_values_in_the_bf16_cache():
     po, pl = oracle.decode(plain)
     np.testing.assert_array_equal(ro, po)
     np.testing.assert_array_equal(rl, pl)
+
+
+# ----------------------------------------------------------------------------- regression guard
+
+def test_oracle_snapshot():
+    """The oracle still produces the values tests/golden/make_oracle_snapshot.py stored
+    (a guard against unintended changes to its arithmetic; correctness is pinned above)."""
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_oracle_snapshot", os.path.join(here, "make_oracle_snapshot.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    stored = json.load(open(os.path.join(here, "oracle_snapshot.json")))
+    now = mod.snapshot()
+    assert set(now) == set(stored["cases"])
+    for name, vals in stored["cases"].items():
+        np.testing.assert_allclose(np.asarray(now[name]["out"]), np.asarray(vals["out"]), rtol=0, atol=1e-12,
+                                   err_msg=name)
+        np.testing.assert_allclose(np.asarray(now[name]["lse"]), np.asarray(vals["lse"]), rtol=0, atol=1e-12,
+                                   err_msg=name)
