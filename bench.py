@@ -593,7 +593,7 @@ def main():
         per["global_decode_b64_paged128_fp8"] = _entry(fd, bd, td, hbm, tf_burst, "inputs larger than L2")
         del w, c8
         torch.cuda.empty_cache()
-        # speculative verification: 4 draft tokens per sequence on the config-3 caches
+        # speculative verification: 4 draft tokens per sequence on the 64-sequence decode caches
         vg, vs = configs.verify(B=64, q_len=4, decode=gl)
         for name, c in (("global_verify_b64_q4", vg), ("swa_verify_b64_q4", vs)):
             fc, bc = chunked_counts(c)

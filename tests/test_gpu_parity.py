@@ -240,7 +240,7 @@ def test_decode_fp8_b64_full_scale():
     seqs = np.array(sorted(set([0, 63] + list(synth.permutation(79, 64)[:6]))))
     ro, rl = oracle.decode(cfg, seqs=seqs)
     idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "fp8 config-3 scale, sampled sequences")
+    parity(out[idx], lse[idx], ro, rl, "fp8 64-sequence decode scale, sampled sequences")
 
 
 @pytest.fixture(scope="module")
@@ -436,7 +436,7 @@ def test_verify_draft_tokens(q_len):
 
 def test_verify_b64_full_scale(dec64):
     """Verification at the decode workload's scale (64 sequences, contexts up to 64K) on the
-    config-3 caches, checked on the rows of 4 sampled sequences."""
+    64-sequence decode caches, checked on the rows of 4 sampled sequences."""
     import torch
     _, gl = dec64
     glb, swa = configs.verify(B=64, q_len=4, decode=gl)
