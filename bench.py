@@ -250,6 +250,67 @@ class Prefill:
                                  workspace=self.ws, kernel_events=kernel_events)
 
 
+class HostPipeline:
+    """End-to-end prefill from pinned host buffers through the C ABI, one call per sequence
+    on the caller's stream: the inputs of later sequences travel host -> device on one copy
+    stream while a sequence computes, and the outputs of earlier ones travel back on another
+    (PCIe carries both directions at once).  Every step copies all of its inputs in and
+    all of its outputs out."""
+
+    def __init__(self, step):
+        import torch
+        cfg = step.cfg
+        if list(cfg.cu_q) != list(cfg.cu_k):
+            raise ValueError("contiguous prefill with as many queries as keys per sequence")
+        self.step, self.M = step, step.M
+        self.cu = [int(x) for x in cfg.cu_q]
+        pin = lambda t: t.cpu().pin_memory()
+        self.q_h, self.k_h, self.v_h, self.s_h = pin(step.q), pin(step.k), pin(step.v), pin(step.sink)
+        self.out_h = torch.empty_like(step.out, device="cpu").pin_memory()
+        self.lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
+        lens = np.diff(np.asarray(self.cu))
+        self.cu1_h = [pin(torch.tensor([0, int(n)], dtype=torch.int32)) for n in lens]
+        self.cu1_d = [torch.empty(2, dtype=torch.int32, device="cuda") for _ in lens]
+        self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def bytes(self):
+        ins = [self.q_h, self.k_h, self.v_h, self.s_h] + self.cu1_h
+        return (sum(t.numel() * t.element_size() for t in ins),
+                sum(t.numel() * t.element_size() for t in (self.out_h, self.lse_h)))
+
+    def __call__(self):
+        import torch
+        st, M, L, cu = self.step, self.M, self.step.cfg.layer, self.cu
+        cur = torch.cuda.current_stream()
+        self.s_in.wait_stream(cur)   # the previous step's calls and copies are done
+        self.s_out.wait_stream(cur)
+        arrived = []
+        with torch.cuda.stream(self.s_in):
+            st.sink.copy_(self.s_h, non_blocking=True)
+            for s in range(len(cu) - 1):
+                a, b = cu[s], cu[s + 1]
+                st.q[a:b].copy_(self.q_h[a:b], non_blocking=True)
+                st.k[a:b].copy_(self.k_h[a:b], non_blocking=True)
+                st.v[a:b].copy_(self.v_h[a:b], non_blocking=True)
+                self.cu1_d[s].copy_(self.cu1_h[s], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_in)
+                arrived.append(ev)
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            cur.wait_event(arrived[s])
+            M.mimo_attn_prefill(st.q[a:b], st.k[a:b], st.v[a:b], self.cu1_d[s], self.cu1_d[s],
+                                num_kv_heads=L.num_kv_heads, rope_base=L.rope_base, window=L.window,
+                                sink=st.sink, out=st.out[a:b], lse=st.lse[a:b], workspace=st.ws)
+            done = torch.cuda.Event()
+            done.record(cur)
+            self.s_out.wait_event(done)
+            with torch.cuda.stream(self.s_out):
+                self.out_h[a:b].copy_(st.out[a:b], non_blocking=True)
+                self.lse_h[a:b].copy_(st.lse[a:b], non_blocking=True)
+        cur.wait_stream(self.s_out)
+
+
 class Decode:
     def __init__(self, cfg):
         import torch
@@ -506,25 +567,10 @@ def main():
             "tensor_frac": flops / (ms_kernel * 1e-3) / 1e12 / tf_burst}
 
     # ---------------- end to end through the C ABI: host buffers, copies inside the timed region
-    q_h = step.q.cpu().pin_memory()
-    k_h, v_h = step.k.cpu().pin_memory(), step.v.cpu().pin_memory()
-    cq_h, ck_h = step.cq.cpu().pin_memory(), step.ck.cpu().pin_memory()
-    s_h = step.sink.cpu().pin_memory()
-    out_h, lse_h = torch.empty_like(step.out, device="cpu").pin_memory(), torch.empty_like(step.lse, device="cpu").pin_memory()
-
-    def e2e_step():
-        step.q.copy_(q_h, non_blocking=True)
-        step.k.copy_(k_h, non_blocking=True)
-        step.v.copy_(v_h, non_blocking=True)
-        step.cq.copy_(cq_h, non_blocking=True)
-        step.ck.copy_(ck_h, non_blocking=True)
-        step.sink.copy_(s_h, non_blocking=True)
-        step()
-        out_h.copy_(step.out, non_blocking=True)
-        lse_h.copy_(step.lse, non_blocking=True)
-
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, cq_h, ck_h, s_h))
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    # (one call per sequence, with the next sequence's inputs and the previous one's outputs
+    # crossing PCIe while a sequence computes)
+    e2e_step = HostPipeline(step)
+    h2d, d2h = e2e_step.bytes()
     for _ in range(2):
         e2e_step()
     ke = max(3, min(args.steps, 10))
@@ -533,8 +579,9 @@ def main():
     if pg:
         te, = max_over_ranks([te], pg, "cuda")
     e2e = {"value": whole_job_rate(flops, world, te) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": te}
-    del q_h, k_h, v_h, out_h, lse_h
+           "d2h_bytes_per_step": d2h, "ms_per_step": te,
+           "method": "pinned host buffers; per-sequence calls with H2D / D2H on two copy streams overlapping the calls"}
+    del e2e_step
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
