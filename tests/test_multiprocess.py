@@ -104,6 +104,40 @@ def test_cp_halo_exchange(splits):
     _run(_cp_worker, len(splits[0]), splits)
 
 
+def _cp_subgroup_worker(rank, world, port):
+    """Ranks 1 and 2 of 3 form the context-parallel group: group ranks map to global ranks."""
+    _init(rank, world, port)
+    try:
+        from global_attention_attn_b200 import cp
+        group = dist.new_group([1, 2])  # every rank takes part in creating it
+        if rank in (1, 2):
+            g = rank - 1
+            lens, starts = [200 if g == 0 else 50], [0 if g == 0 else 200]
+            recv_k, recv_v = cp.ring_buffers(1, 1, "cpu", torch.float32)
+            send_k, send_v = cp.ring_buffers(1, 1, "cpu", torch.float32)
+
+            def fill(rk, rv):
+                for _, pos0, m in cp.tail_ranges(lens, starts):
+                    for p in range(pos0, pos0 + m):
+                        rk[0, p % RING] = _marker(0, p)
+                        rv[0, p % RING] = -_marker(0, p)
+
+            cp.exchange_halo(send_k, send_v, recv_k, recv_v, fill, independent=cp.chunks_fill_ring(lens), group=group)
+            if g == 1:  # positions 72..199 from group rank 0
+                for slot in range(RING):
+                    p = 200 - RING + (slot - (200 - RING)) % RING
+                    assert torch.all(recv_k[0, slot] == _marker(0, p)), (slot, p)
+            else:
+                assert torch.all(recv_k == 0)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cp_halo_exchange_in_a_subgroup():
+    _run(_cp_subgroup_worker, 3)
+
+
 # ----------------------------------------------------------------------------- CP host logic
 
 def test_cp_tail_ranges_and_modes():
