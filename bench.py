@@ -36,12 +36,13 @@ from workloads import configs  # noqa: E402
 METRIC = "SWA+sink / global attn prefill TFLOP/s, decode KV GB/s; % of B200 roofline"
 FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) pair
 
-# The step's dominant kernel (about 97% of the step's device time in the ncu launch list).
+# The step's dominant kernel (about 96% of the step's device time in the ncu launch list).
 DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
-# workload, from the ncu capture summarised in profiles/prefill_swa_kernel_2x4096_full.md
-# (kernel at commit 4bd734f): 249.66 MB read + 104.12 MB written for 2 x 4096 tokens, scaled
-# by tokens to the 40696-token workload.  Removed whenever the kernel changes.
+# workload.  Measured with one ncu capture of the kernel on a 2 x 4096-token sliding-window
+# prefill (inputs larger than L2): 249.66 MB read + 104.12 MB written, scaled by tokens to the
+# 40696-token workload (the kernel's traffic is proportional to tokens).  Set to None whenever
+# the kernel changes after the capture.
 TRAFFIC_BYTES = {"prefill_swa_kernel": int((249.656832e6 + 104.123392e6) * 40696 / 8192)}
 
 
@@ -614,7 +615,7 @@ def main():
         for _ in range(3):
             w2()
         t2 = event_time_ms(w2, 10) / 10
-        per["global_prefill_s16384"] = _entry(f2, b2, t2, hbm, tf_sust, "inputs larger than L2")
+        per["global_prefill_s16384"] = _entry(f2, b2, t2, hbm, tf_burst, "inputs larger than L2")
         del w2, c2
         torch.cuda.empty_cache()
         sw, gl = configs.decode_batch()
@@ -659,7 +660,7 @@ def main():
             for _ in range(3):
                 w()
             tc = event_time_ms(w, 5) / 5
-            per[name] = _entry(fc, bc, tc, hbm, tf_sust if c.paged else tf_burst, "inputs larger than L2")
+            per[name] = _entry(fc, bc, tc, hbm, tf_burst, "inputs larger than L2")
             del w
         line["per_config"] = per
         line["cpu_baseline"] = cpu_baseline(cfg)

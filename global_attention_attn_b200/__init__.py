@@ -22,11 +22,15 @@ MIMO_ERR_CUDA = 4
 MIMO_ERR_TIMEOUT = 5
 MIMO_STATUS_TIMEOUT = 1
 MIMO_STATUS_BAD_INDEX = 2
+MIMO_STATUS_RANGE = 4
+MIMO_STATUS_BAD_SCALE = 8
 MIMO_CACHE_NONE = 0
 MIMO_CACHE_PAGED = 1
 MIMO_CACHE_RING = 2
 MIMO_DTYPE_BF16 = 0
 MIMO_DTYPE_FP8_E4M3 = 1
+MIMO_RING_SLOTS_DEFAULT = 128
+MIMO_RING_SLOTS_MAX = 512
 
 NUM_Q_HEADS = 64
 HEAD_DIM_QK = 192
@@ -35,7 +39,7 @@ ROPE_DIM = 64
 SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
 V_SCALE = 0.707
 
-EXPORTS = ("mimo_attn_prefill", "mimo_attn_prefill_workspace_size", "mimo_attn_decode",
+EXPORTS = ("mimo_attn_prefill", "mimo_attn_prefill_workspace_size", "mimo_attn_prefill_stall_test", "mimo_attn_decode",
            "mimo_attn_decode_workspace_size", "mimo_attn_decode_noalloc", "mimo_kv_append", "mimo_last_error",
            "mimo_status_poll", "mimo_version", "mimo_window_from_left_right")
 DECODE_NOALLOC_MAX_BYTES = 16 << 20
@@ -55,7 +59,8 @@ class MimoPrefillArgs(C.Structure):
                 ("q", _P), ("k", _P), ("v", _P), ("cu_seqlens_q", _P), ("cu_seqlens_k", _P), ("cache_lens", _P),
                 ("cache_kind", C.c_int), ("k_cache", _P), ("v_cache", _P), ("block_table", _P),
                 ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P), ("workspace", _P),
-                ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P), ("ev_kernel_end", _P)]
+                ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P), ("ev_kernel_end", _P),
+                ("ring_slots", C.c_int)]
 
 
 class MimoDecodeArgs(C.Structure):
@@ -63,7 +68,8 @@ class MimoDecodeArgs(C.Structure):
                 ("seq_lens", _P), ("cache_kind", C.c_int), ("k_cache", _P), ("v_cache", _P),
                 ("block_table", _P), ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P),
                 ("workspace", _P), ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P),
-                ("ev_kernel_end", _P), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P)]
+                ("ev_kernel_end", _P), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P),
+                ("ring_slots", C.c_int)]
 
 
 class MimoAppendArgs(C.Structure):
@@ -71,7 +77,8 @@ class MimoAppendArgs(C.Structure):
                 ("head_dim_v", C.c_int), ("rope_dim", C.c_int), ("rope_base", C.c_double), ("k_new", _P),
                 ("v_new", _P), ("pos", _P), ("seq_idx", _P), ("cache_kind", C.c_int), ("k_cache", _P),
                 ("v_cache", _P), ("num_seqs", C.c_int), ("block_table", _P), ("max_pages", C.c_int),
-                ("num_pages", C.c_int), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P)]
+                ("num_pages", C.c_int), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P),
+                ("ring_slots", C.c_int)]
 
 
 _lib = None
@@ -95,6 +102,8 @@ def lib():
         L.mimo_attn_prefill.restype = C.c_int
         L.mimo_attn_prefill_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]
         L.mimo_attn_prefill_workspace_size.restype = C.c_size_t
+        L.mimo_attn_prefill_stall_test.argtypes = [C.POINTER(MimoPrefillArgs), _P, C.c_ulonglong]
+        L.mimo_attn_prefill_stall_test.restype = C.c_int
         L.mimo_attn_decode.argtypes = [C.POINTER(MimoDecodeArgs), _P]
         L.mimo_attn_decode.restype = C.c_int
         L.mimo_attn_decode_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
@@ -163,10 +172,13 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
                       sink=None, cache_lens=None, cache_kind: int = MIMO_CACHE_NONE, k_cache=None, v_cache=None,
                       block_table=None, num_pages: int = 0, out=None, lse=None, workspace=None,
                       softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None,
-                      with_lse: bool = True, kernel_events=None):
+                      with_lse: bool = True, kernel_events=None, ring_slots: int = 0,
+                      stall_test_wait_ns: int | None = None):
     """Varlen prefill (see include/mimoattn.h).  Tensors are CUDA tensors: q/k/v/caches bf16,
     index tensors int32, sink fp32.  kernel_events: optional (begin, end) pair of recorded-once
-    torch.cuda.Event placed around the attention kernel.  Returns (out, lse)."""
+    torch.cuda.Event placed around the attention kernel.  ring_slots: slots per sequence of a
+    ring cache (0 = 128).  stall_test_wait_ns: call mimo_attn_prefill_stall_test instead (the
+    failure-detection test whose waits run out after that many ns).  Returns (out, lse)."""
     import torch
     total_q = q.shape[0]
     num_seqs = cu_seqlens_q.shape[0] - 1
@@ -191,7 +203,11 @@ def mimo_attn_prefill(q, k, v, cu_seqlens_q, cu_seqlens_k, *, num_kv_heads: int,
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
-    _check(lib().mimo_attn_prefill(C.byref(a), _stream(stream)))
+    a.ring_slots = int(ring_slots)
+    if stall_test_wait_ns is not None:
+        _check(lib().mimo_attn_prefill_stall_test(C.byref(a), _stream(stream), int(stall_test_wait_ns)))
+    else:
+        _check(lib().mimo_attn_prefill(C.byref(a), _stream(stream)))
     return out, lse
 
 
@@ -199,9 +215,10 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
                      cache_kind: int, k_cache, v_cache, block_table=None, num_pages: int = 0, sink=None, out=None,
                      lse=None, workspace=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE,
                      stream=None, with_lse: bool = True, kernel_events=None, cache_dtype: int = MIMO_DTYPE_BF16,
-                     k_dequant=None, v_dequant=None):
+                     k_dequant=None, v_dequant=None, ring_slots: int = 0):
     """Decode step (see include/mimoattn.h).  kernel_events as for mimo_attn_prefill (around the
-    split kernel, not the combine).  Returns (out, lse)."""
+    split kernel, not the combine).  ring_slots: slots per sequence of a ring cache (0 = 128).
+    Returns (out, lse)."""
     import torch
     B = q.shape[0]
     if out is None:
@@ -224,6 +241,7 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
     a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
+    a.ring_slots = int(ring_slots)
     _check(lib().mimo_attn_decode(C.byref(a), _stream(stream)))
     return out, lse
 
@@ -231,7 +249,7 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
 def mimo_attn_decode_noalloc(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_base: float, window: int,
                              cache_kind: int, k_cache, v_cache, out, lse=None, block_table=None, num_pages: int = 0,
                              sink=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE, stream=None,
-                             cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None):
+                             cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None, ring_slots: int = 0):
     """Decode that allocates nothing (see mimo_attn_decode_noalloc in include/mimoattn.h): the
     caller passes the output buffers; the split-KV partials go to the library's static
     device scratch (16 MiB), so concurrent calls must not overlap on the GPU."""
@@ -245,15 +263,17 @@ def mimo_attn_decode_noalloc(q, seq_lens, *, max_seq_len: int, num_kv_heads: int
     a.num_pages = num_pages
     a.out, a.lse = _ptr(out), _ptr(lse)
     a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
+    a.ring_slots = int(ring_slots)
     _check(lib().mimo_attn_decode_noalloc(C.byref(a), _stream(stream)))
     return out, lse
 
 
 def mimo_kv_append(k_new, v_new, pos, seq_idx, *, rope_base: float, cache_kind: int, k_cache, v_cache,
                    num_seqs: int, block_table=None, num_pages: int = 0, stream=None,
-                   cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None):
+                   cache_dtype: int = MIMO_DTYPE_BF16, k_dequant=None, v_dequant=None, ring_slots: int = 0):
     """Rotate and store new keys/values into the ring or paged cache (see include/mimoattn.h);
-    an E4M3 cache (cache_dtype) quantises with the per-KV-head scales k_dequant / v_dequant."""
+    an E4M3 cache (cache_dtype) quantises with the per-KV-head scales k_dequant / v_dequant.
+    ring_slots: slots per sequence of a ring cache (0 = 128)."""
     a = MimoAppendArgs()
     a.num_tokens, a.num_kv_heads = k_new.shape[0], k_new.shape[1]
     a.head_dim_qk, a.head_dim_v, a.rope_dim, a.rope_base = HEAD_DIM_QK, HEAD_DIM_V, ROPE_DIM, float(rope_base)
@@ -265,6 +285,7 @@ def mimo_kv_append(k_new, v_new, pos, seq_idx, *, rope_base: float, cache_kind: 
     a.max_pages = 0 if block_table is None else block_table.shape[1]
     a.num_pages = num_pages
     a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
+    a.ring_slots = int(ring_slots)
     _check(lib().mimo_kv_append(C.byref(a), _stream(stream)))
 
 

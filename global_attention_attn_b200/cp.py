@@ -139,17 +139,29 @@ def swa_prefill_context_parallel(q, k, v, chunk_lens: Sequence[int], start_pos: 
     (host integers) give each chunk's length and first position.  Rank r's chunk of a
     sequence starts where rank r - 1's ends, and rank 0's at position 0.  Returns
     (out, lse) for the local rows."""
+    import contextlib
+
     import torch.distributed as dist
     if dist.get_rank(group) == 0 and any(int(p) != 0 for p in start_pos):
         raise ValueError("rank 0 holds the first chunk of every sequence (start position 0)")
     rope_base = float(rope_base)
     num_seqs, hkv = len(chunk_lens), k.shape[1]
-    recv_k, recv_v = ring_buffers(num_seqs, hkv, q.device)
-    send_k, send_v = ring_buffers(num_seqs, hkv, q.device)
+    # torch.distributed orders its transfers against the current stream, so every step
+    # (zeroing the rings, the appends, the send / receive, the prefill) runs with `stream`
+    # made current: the send then follows the append that fills the ring, and the prefill
+    # follows the receive.  The caller orders q / k / v against `stream`.
+    if stream is not None:
+        import torch
+        scope = torch.cuda.stream(stream)
+    else:
+        scope = contextlib.nullcontext()
+    with scope:
+        recv_k, recv_v = ring_buffers(num_seqs, hkv, q.device)
+        send_k, send_v = ring_buffers(num_seqs, hkv, q.device)
 
-    def fill(rk, rv):
-        fill_ring_tail(rk, rv, k, v, chunk_lens, start_pos, rope_base=rope_base, stream=stream)
+        def fill(rk, rv):
+            fill_ring_tail(rk, rv, k, v, chunk_lens, start_pos, rope_base=rope_base)
 
-    exchange_halo(send_k, send_v, recv_k, recv_v, fill, independent=chunks_fill_ring(chunk_lens), group=group)
-    return prefill_with_halo(q, k, v, chunk_lens, start_pos, recv_k, recv_v, rope_base=rope_base, window=window,
-                             sink=sink, out=out, lse=lse, stream=stream)
+        exchange_halo(send_k, send_v, recv_k, recv_v, fill, independent=chunks_fill_ring(chunk_lens), group=group)
+        return prefill_with_halo(q, k, v, chunk_lens, start_pos, recv_k, recv_v, rope_base=rope_base,
+                                 window=window, sink=sink, out=out, lse=lse)

@@ -18,6 +18,10 @@ namespace mimo {
 
 __device__ unsigned g_status_word;
 
+// Split-KV partials of mimo_attn_decode_noalloc.  Device code never names it: host code
+// passes the per-device address that dev_state() looks up.
+static __device__ __align__(256) unsigned char g_decode_scratch[MIMO_DECODE_NOALLOC_MAX_BYTES];
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -60,10 +64,40 @@ RopeFreqs make_freqs(double base) {
   return f;
 }
 
-// Per-device state: address of the status word and the SM count.
+// Id of the calling thread's current CUDA context (0 if none), through the driver entry
+// points the runtime exposes: a context that was destroyed and re-created (a device reset)
+// gets a new id, and its module globals new addresses.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Per-device state: addresses of the status word and of the no-alloc decode scratch in
+// this device's copy of the module, the SM count, and the context they belong to.  Looked
+// up on the first call on a device (with that device current) and again whenever the
+// current context is not the one they were looked up in.
 struct DevState {
   unsigned* status = nullptr;
+  void* scratch = nullptr;
   int sms = 0;
+  unsigned long long ctx = 0;
 };
 std::mutex g_mu;
 DevState g_dev[64];
@@ -75,15 +109,37 @@ int dev_state(const char* fn, DevState* out) {
   if (dev < 0 || dev >= 64) return fail(MIMO_ERR_CUDA, "%s: device index %d out of range", fn, dev);
   std::lock_guard<std::mutex> lk(g_mu);
   DevState& d = g_dev[dev];
-  if (!d.status) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_status_word);
-    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress: %s", fn, cudaGetErrorString(e));
-    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (!d.status || d.ctx != current_ctx_id()) {
+    // cudaGetSymbolAddress makes the device's primary context current (creating it if
+    // needed), so the context id is read after it.
+    void* st = nullptr;
+    void* sc = nullptr;
+    e = cudaGetSymbolAddress(&st, g_status_word);
+    if (e != cudaSuccess || !st)
+      return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress (status word): %s", fn, cudaGetErrorString(e));
+    e = cudaGetSymbolAddress(&sc, g_decode_scratch);
+    if (e != cudaSuccess || !sc)
+      return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress (decode scratch): %s", fn, cudaGetErrorString(e));
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaDeviceGetAttribute: %s", fn, cudaGetErrorString(e));
-    d.status = static_cast<unsigned*>(ptr);
+    d.status = static_cast<unsigned*>(st);
+    d.scratch = sc;
+    d.sms = sms;
+    d.ctx = current_ctx_id();
   }
   *out = d;
+  return MIMO_OK;
+}
+
+// Slots per sequence of a ring cache: 0 means the default; else a multiple of the 16-key
+// tile in [128, 512].
+int ring_slots_of(const char* fn, int v, int* out) {
+  if (v == 0) v = MIMO_RING_SLOTS_DEFAULT;
+  if (v < MIMO_RING_SLOTS_DEFAULT || v > MIMO_RING_SLOTS_MAX || v % 16)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: ring_slots must be 0 (128) or a multiple of 16 in 128..512 (got %d)", fn,
+                v);
+  *out = v;
   return MIMO_OK;
 }
 
@@ -214,9 +270,12 @@ int mimo_kv_append(const mimo_append_args* a, void* stream) {
       return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages and num_pages must be > 0 for a paged cache", fn);
   }
   if (int rc = check_cache_dtype(fn, a->cache_dtype, a->k_dequant, a->v_dequant)) return rc;
+  int ring_slots = 0;
+  if (int rc = ring_slots_of(fn, a->ring_slots, &ring_slots)) return rc;
   DevState d;
   if (int rc = dev_state(fn, &d)) return rc;
   AppendParams p;
+  p.ring_slots = ring_slots;
   p.num_tokens = a->num_tokens;
   p.hkv = a->num_kv_heads;
   p.k_new = static_cast<const uint16_t*>(a->k_new);
@@ -249,8 +308,11 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   if (a->max_seq_len <= 0) return fail(MIMO_ERR_INVALID_ARG, "%s: max_seq_len must be > 0", fn);
   if (a->cache_kind != MIMO_CACHE_RING && a->cache_kind != MIMO_CACHE_PAGED)
     return fail(MIMO_ERR_INVALID_ARG, "%s: cache_kind must be MIMO_CACHE_RING or MIMO_CACHE_PAGED", fn);
-  if (a->cache_kind == MIMO_CACHE_RING && (a->layer.window <= 0 || a->layer.window > 128))
-    return fail(MIMO_ERR_INVALID_ARG, "%s: a ring cache holds 128 positions: window must be in 1..128", fn);
+  int ring_slots = 0;
+  if (int rc = ring_slots_of(fn, a->ring_slots, &ring_slots)) return rc;
+  if (a->cache_kind == MIMO_CACHE_RING && (a->layer.window <= 0 || a->layer.window > ring_slots))
+    return fail(MIMO_ERR_INVALID_ARG, "%s: a ring cache of %d slots holds %d positions: window must be in 1..%d", fn,
+                ring_slots, ring_slots, ring_slots);
   REQUIRE_PTR(a->q, "q");
   REQUIRE_PTR(a->seq_lens, "seq_lens");
   REQUIRE_PTR(a->k_cache, "k_cache");
@@ -280,7 +342,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   {
-    const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * kPage : long(a->num_pages) * kPage;
+    const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * ring_slots : long(a->num_pages) * kPage;
     const bool fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
     int rc = make_map(fn, enc, &p.tm_q, a->q, a->batch, kHq, kDqk, 16, 1);
     if (!rc) rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 16, fp8);
@@ -300,6 +362,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   p.q = static_cast<const uint16_t*>(a->q);
   p.seq_lens = a->seq_lens;
   p.cache_kind = a->cache_kind;
+  p.ring_slots = ring_slots;
   p.k_cache = static_cast<const uint16_t*>(a->k_cache);
   p.v_cache = static_cast<const uint16_t*>(a->v_cache);
   p.block_table = a->block_table;
@@ -321,8 +384,16 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   return MIMO_OK;
 }
 
-int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
-  const char* fn = "mimo_attn_prefill";
+}  // extern "C"
+
+namespace mimo {
+namespace {
+
+// Every bounded wait of the kernels gives up after this long by default.
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsigned long long wait_ns,
+                 int withhold_q) {
   if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
   if (int rc = check_layer(fn, a->layer)) return rc;
   if (a->num_seqs <= 0) return fail(MIMO_ERR_INVALID_ARG, "%s: num_seqs must be > 0", fn);
@@ -336,7 +407,8 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   if (a->lse && (reinterpret_cast<uintptr_t>(a->lse) & 3))
     return fail(MIMO_ERR_INVALID_ARG, "%s: lse is not 4-byte aligned", fn);
   const int hkv = a->layer.num_kv_heads;
-  int mode;
+  int mode, ring_slots = 0;
+  if (int rc = ring_slots_of(fn, a->ring_slots, &ring_slots)) return rc;
   if (a->cache_kind == MIMO_CACHE_PAGED) {
     if (a->k || a->v || a->cu_seqlens_k || a->total_k)
       return fail(MIMO_ERR_INVALID_ARG,
@@ -440,6 +512,8 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   p.lse = a->lse;
   p.rope = make_freqs(a->layer.rope_base);
   p.status = d.status;
+  p.wait_ns = wait_ns;
+  p.withhold_q = withhold_q;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode != kModePaged) {
@@ -454,6 +528,7 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
     r.v = static_cast<const uint16_t*>(a->v);
     r.ring_k = static_cast<const uint16_t*>(a->k_cache);
     r.ring_v = static_cast<const uint16_t*>(a->v_cache);
+    r.ring_slots = ring_slots;
     r.ws_k = ws_k;
     r.ws_v = ws_v;
     r.total_q = kind == 0 ? a->total_q : 0;
@@ -490,39 +565,23 @@ int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
   return MIMO_OK;
 }
 
-}  // extern "C"
-
-namespace mimo {
-namespace {
-
-// Split-KV partials of mimo_attn_decode_noalloc.  Device code never names it:
-// host code passes the per-device address obtained below.
-static __device__ __align__(256) unsigned char g_decode_scratch[MIMO_DECODE_NOALLOC_MAX_BYTES];
-
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[64];
-
-// Address of this device's copy of g_decode_scratch (looked up once per device,
-// with that device current).  In host code the array's name is only a stand-in.
-int scratch_address(const char* fn, void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
-  if (dev < 0 || dev >= 64) return fail(MIMO_ERR_CUDA, "%s: device index %d out of range", fn, dev);
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    if (e != cudaSuccess || !ptr)
-      return fail(MIMO_ERR_CUDA, "%s: cudaGetSymbolAddress of the scratch array: %s", fn, cudaGetErrorString(e));
-    g_scratch_ptr[dev] = ptr;
-  }
-  *out = g_scratch_ptr[dev];
-  return MIMO_OK;
-}
-
 }  // namespace
 }  // namespace mimo
+
+extern "C" {
+
+int mimo_attn_prefill(const mimo_prefill_args* a, void* stream) {
+  return prefill_impl("mimo_attn_prefill", a, stream, kWaitNs, 0);
+}
+
+int mimo_attn_prefill_stall_test(const mimo_prefill_args* a, void* stream, unsigned long long wait_limit_ns) {
+  const char* fn = "mimo_attn_prefill_stall_test";
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > 10000000000ull)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: wait_limit_ns must be in 1e6..1e10 (got %llu)", fn, wait_limit_ns);
+  return prefill_impl(fn, a, stream, wait_limit_ns, 1);
+}
+
+}  // extern "C"
 
 extern "C" {
 
@@ -542,7 +601,10 @@ int mimo_attn_decode_noalloc(const mimo_decode_args* a, void* stream) {
   b.workspace = nullptr;
   b.workspace_bytes = 0;
   if (a->batch > 0) {
-    if (int rc = scratch_address(fn, &b.workspace)) return rc;
+    // this device's copy of the static array (in host code its name is only a stand-in)
+    DevState d;
+    if (int rc = dev_state(fn, &d)) return rc;
+    b.workspace = d.scratch;
     b.workspace_bytes = MIMO_DECODE_NOALLOC_MAX_BYTES;
   }
   return mimo_attn_decode(&b, stream);

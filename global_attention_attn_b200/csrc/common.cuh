@@ -21,6 +21,19 @@ __device__ __forceinline__ uint32_t pack2_f16(float lo, float hi) {
   return uint32_t(__half_as_ushort(__float2half_rn(lo))) | (uint32_t(__half_as_ushort(__float2half_rn(hi))) << 16);
 }
 
+// Largest finite fp16 value.  The rotated query / key dims are kept in fp16; a component
+// beyond it is stored as +-65504 and reported with MIMO_STATUS_RANGE.
+constexpr float kF16Max = 65504.f;
+
+// Two floats -> fp16x2 rounded to nearest even, saturating at +-65504 (NaN stays NaN);
+// `amax` collects the largest magnitude seen so that the caller can report saturation.
+__device__ __forceinline__ uint32_t pack2_f16_sat(float lo, float hi, float& amax) {
+  uint32_t d;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+  return d;
+}
+
 // cos / sin of pos * inv_freq.  The angle and its reduction to [-pi, pi] are
 // taken in float64 (the fastest rotary angle equals the position, up to ~1.3e5
 // radians here, far past where a float32 angle keeps its digits); only the
@@ -52,8 +65,10 @@ __device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t x) {
 // dims 8u+32..8u+39 (u in 0..3); frequency index of element i is 8u+i.
 // Input bf16, output IEEE fp16: the rotated dims are kept in fp16 everywhere
 // (query tiles, key copies, caches) because their rounding error enters every
-// logit; fp16 has 11 significant bits against bf16's 8.
-__device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int pos, const RopeFreqs& rf) {
+// logit; fp16 has 11 significant bits against bf16's 8.  Outputs saturate at
+// +-65504 and `amax` collects the largest magnitude (see pack2_f16_sat).
+__device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int pos, const RopeFreqs& rf,
+                                                float& amax) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
@@ -63,13 +78,13 @@ __device__ __forceinline__ void rope_chunk_pair(uint4& lo, uint4& hi, int u, int
     float c0, s0, c1, s1;
     rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w], &c0, &s0);
     rope_cos_sin(pos, rf.inv_freq[8 * u + 2 * w + 1], &c1, &s1);
-    a[w] = pack2_f16(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
-    b[w] = pack2_f16(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1);
+    a[w] = pack2_f16_sat(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1, amax);
+    b[w] = pack2_f16_sat(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1, amax);
   }
 }
 
 // Same rotation with precomputed (cos, sin) pairs: cs[i] for frequency 8u+i.
-__device__ __forceinline__ void rope_chunk_pair_cs(uint4& lo, uint4& hi, const float2* cs) {
+__device__ __forceinline__ void rope_chunk_pair_cs(uint4& lo, uint4& hi, const float2* cs, float& amax) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
@@ -77,14 +92,14 @@ __device__ __forceinline__ void rope_chunk_pair_cs(uint4& lo, uint4& hi, const f
     const float x0 = lo_bf16(a[w]), x1 = hi_bf16(a[w]);
     const float y0 = lo_bf16(b[w]), y1 = hi_bf16(b[w]);
     const float2 t0 = cs[2 * w], t1 = cs[2 * w + 1];
-    a[w] = pack2_f16(x0 * t0.x - y0 * t0.y, x1 * t1.x - y1 * t1.y);
-    b[w] = pack2_f16(y0 * t0.x + x0 * t0.y, y1 * t1.x + x1 * t1.y);
+    a[w] = pack2_f16_sat(x0 * t0.x - y0 * t0.y, x1 * t1.x - y1 * t1.y, amax);
+    b[w] = pack2_f16_sat(y0 * t0.x + x0 * t0.y, y1 * t1.x + x1 * t1.y, amax);
   }
 }
 
 // Same rotation on packed fp32 pairs: cs[w] = (cos_a, sin_a, cos_b, sin_b) for the
 // two frequencies held by 32-bit word w of the chunks.
-__device__ __forceinline__ void rope_chunk_pair_cs4(uint4& lo, uint4& hi, const float4* cs) {
+__device__ __forceinline__ void rope_chunk_pair_cs4(uint4& lo, uint4& hi, const float4* cs, float& amax) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
@@ -104,8 +119,8 @@ __device__ __forceinline__ void rope_chunk_pair_cs4(uint4& lo, uint4& hi, const 
     float a0, a1, b0, b1;
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(r0));
     asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(r1));
-    a[w] = pack2_f16(a0, a1);
-    b[w] = pack2_f16(b0, b1);
+    a[w] = pack2_f16_sat(a0, a1, amax);
+    b[w] = pack2_f16_sat(b0, b1, amax);
   }
 }
 

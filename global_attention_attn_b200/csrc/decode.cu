@@ -107,7 +107,7 @@ __device__ __forceinline__ bool unit_at(const DecodeParams& p, int u, UnitInfo& 
   U.k_end = min(U.k_begin + p.split_len, U.ctx);
   if (p.cache_kind == MIMO_CACHE_RING) {
     U.t0 = 0;
-    U.nt = kPage / kTileK;  // the 128 slots, in slot order
+    U.nt = p.ring_slots / kTileK;  // every slot of the ring, in slot order
   } else {
     U.t0 = U.k_begin / kTileK;
     U.nt = (U.k_end - 1) / kTileK - U.t0 + 1;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       for (int t = 0; t < U.nt; ++t, ++it) {
         int row;
         if (p.cache_kind == MIMO_CACHE_RING) {
-          row = U.s * kPage + kTileK * t;
+          row = U.s * p.ring_slots + kTileK * t;
         } else {
           const int key = (U.t0 + t) * kTileK;
           row = __shfl_sync(0xffffffffu, row_l, key / kPage - p0) + key % kPage;
@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               t0 = I->t0;
     // ---- query fragments (A of m16n8k16) from the swizzled tile; rows = heads of the group
     uint32_t qa[12][4];
+    float q_amax = 0.f;  // largest rotated (or, for E4M3, converted) query component
     const float4* cs = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(I + 1));
     const uint32_t qt = qtile0 + b * kQBytes;
     if constexpr (!FP8) {
@@ -345,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const float4 t = cs[j0 >> 1];  // (cos, sin) of frequencies j0, j0 + 1
           const uint32_t xw = qa[kk][e], yw = qa[kk + 2][e];
           const float x0 = lo_bf16(xw), x1 = hi_bf16(xw), y0 = lo_bf16(yw), y1 = hi_bf16(yw);
-          qa[kk][e] = pack2_f16(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-          qa[kk + 2][e] = pack2_f16(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+          qa[kk][e] = pack2_f16_sat(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w, q_amax);
+          qa[kk + 2][e] = pack2_f16_sat(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w, q_amax);
         }
     } else {
       // E4M3 keys are read with ldmatrix as pairs of bytes, which gives thread (r0, q4) the
@@ -373,14 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const float4 t = cs[j0 >> 1];
           const uint32_t xw = qa[kk][e], yw = qa[kk + 2][e];
           const float x0 = lo_bf16(xw), x1 = hi_bf16(xw), y0 = lo_bf16(yw), y1 = hi_bf16(yw);
-          qa[kk][e] = pack2_f16(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w);
-          qa[kk + 2][e] = pack2_f16(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w);
+          qa[kk][e] = pack2_f16_sat(x0 * t.x - y0 * t.y, x1 * t.z - y1 * t.w, q_amax);
+          qa[kk + 2][e] = pack2_f16_sat(y0 * t.x + x0 * t.y, y1 * t.z + x1 * t.w, q_amax);
         }
 #pragma unroll
       for (int kk = 4; kk < 12; ++kk)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) qa[kk][e] = pack2_f16(lo_bf16(qa[kk][e]), hi_bf16(qa[kk][e]));
+        for (int e = 0; e < 4; ++e) qa[kk][e] = pack2_f16_sat(lo_bf16(qa[kk][e]), hi_bf16(qa[kk][e]), q_amax);
     }
+    if (q_amax > kF16Max) atomicOr(status, MIMO_STATUS_RANGE);
     __syncwarp();
     if (lane == 0) mbar_arrive(q_empty(b));
     const float c_log2 = FP8 ? p.scale_log2 * p.k_dequant[g] : p.scale_log2;
@@ -453,9 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int col = ((e & 2) ? 8 : 0) + 2 * q4 + (e & 1);  // within the 16-key tile
         int kp;
         if (p.cache_kind == MIMO_CACHE_RING) {
-          const int slot = kTileK * t + col;
-          const int base = ctx - kPage;  // the ring holds positions base .. ctx-1
-          kp = base + (((slot - base) % kPage) + kPage) % kPage;
+          const int slot = kTileK * t + col, R = p.ring_slots;
+          const int base = ctx - R;  // the ring holds positions base .. ctx-1
+          kp = base + (((slot - base) % R) + R) % R;
         } else {
           kp = (t0 + t) * kTileK + col;
         }

@@ -12,7 +12,7 @@ constexpr int kDqk = 192;
 constexpr int kDv = 128;
 constexpr int kRope = 64;
 constexpr int kHalf = kRope / 2;
-constexpr int kPage = 128;  // positions per page / ring slots
+constexpr int kPage = 128;  // positions per page (and the default ring slots)
 
 // Rotary frequencies base^(-2j/64), j = 0..31, evaluated on the host in float64.
 struct RopeFreqs {
@@ -29,6 +29,7 @@ struct AppendParams {
   uint16_t* k_cache;
   uint16_t* v_cache;
   int num_seqs;
+  int ring_slots;            // ring: slots per sequence
   const int32_t* block_table;
   int max_pages, num_pages;
   int fp8;                   // cache rows hold E4M3 bytes (quantised by 1 / k_dequant[g], 1 / v_dequant[g])
@@ -51,6 +52,7 @@ struct DecodeParams {
   const uint16_t* q;
   const int32_t* seq_lens;
   int cache_kind;
+  int ring_slots;  // ring: slots per sequence (a multiple of the 16-key tile)
   const uint16_t* k_cache;
   const uint16_t* v_cache;
   const int32_t* block_table;
@@ -93,6 +95,8 @@ struct PrefillParams {
   float* lse;
   RopeFreqs rope;
   unsigned* status;
+  unsigned long long wait_ns;  // limit of every bounded wait in the kernel
+  int withhold_q;              // failure-detection test: the producer never loads a query tile
 };
 
 // Pre-pass of the prefill: rotated key copies into the workspace.
@@ -102,8 +106,9 @@ struct RopeKParams {
   const int32_t* cache_lens;
   const uint16_t* k;
   const uint16_t* v;
-  const uint16_t* ring_k;  // ext mode
+  const uint16_t* ring_k;  // ext mode: [num_seqs, ring_slots, hkv, D]
   const uint16_t* ring_v;
+  int ring_slots;
   uint16_t* ws_k;  // contig: [total_k, hkv, 64]; ext: [total_k + 128*B, hkv, 192]
   uint16_t* ws_v;  // ext: [total_k + 128*B, hkv, 128]
   // per-query-row (cos, sin) of the 32 rotary frequencies, or null

@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     return;
   }
   if (p.cache_kind == MIMO_CACHE_RING) {
-    entry = long(s) * kPage + (pos % kPage);
+    entry = long(s) * p.ring_slots + (pos % p.ring_slots);
   } else {
     const int pi = pos / kPage;
     const int page = pi < p.max_pages ? p.block_table[long(s) * p.max_pages + pi] : -1;
@@ -40,8 +40,14 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   const uint4* ks = reinterpret_cast<const uint4*>(p.k_new + (long(t) * p.hkv + g) * kDqk);
   if (p.fp8) {
     // E4M3 rows: each element divided by its KV head's dequantisation scale, rounded to
-    // nearest even and saturated (the rotation itself in fp32)
-    const float kq = 1.f / p.k_dequant[g], vq = 1.f / p.v_dequant[g];
+    // nearest even and saturated (the rotation itself in fp32).  A scale that is not finite
+    // and positive would store inf / NaN or sign-flipped codes: skip the row and report it.
+    const float kdq = p.k_dequant[g], vdq = p.v_dequant[g];
+    if (!(kdq > 0.f && kdq < INFINITY && vdq > 0.f && vdq < INFINITY)) {
+      if (lane == 0) atomicOr(p.status, MIMO_STATUS_BAD_SCALE);
+      return;
+    }
+    const float kq = 1.f / kdq, vq = 1.f / vdq;
     uint8_t* k8 = reinterpret_cast<uint8_t*>(p.k_cache) + (entry * p.hkv + g) * kDqk;
     uint8_t* v8 = reinterpret_cast<uint8_t*>(p.v_cache) + (entry * p.hkv + g) * kDv;
     auto pack8 = [](const float* x, float sc) {
@@ -85,7 +91,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   uint4* kd = reinterpret_cast<uint4*>(p.k_cache + (entry * p.hkv + g) * kDqk);
   if (lane < 4) {
     uint4 lo = __ldg(ks + lane), hi = __ldg(ks + lane + 4);
-    rope_chunk_pair(lo, hi, lane, pos, p.rope);
+    float amax = 0.f;
+    rope_chunk_pair(lo, hi, lane, pos, p.rope, amax);
+    if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
     kd[lane] = lo;
     kd[lane + 4] = hi;
   } else if (lane >= 8 && lane < 24) {

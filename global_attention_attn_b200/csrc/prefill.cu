@@ -287,8 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         TileInfo T;
         if (!locate<KIND>(p, S, w, T)) break;
         if (lane == 0) {
+          if (p.withhold_q) break;  // failure-detection test: no query tile ever arrives
           const int qs = mt % NQ;
-          if (mt >= NQ) ok = mbar_wait(q_empty(qs), ((mt / NQ) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+          if (mt >= NQ) ok = mbar_wait(q_empty(qs), ((mt / NQ) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns);
           if (!ok) break;
           const uint32_t qdst = sbase + Ly::kOffQ + qs * Ly::kQStage;
           mbar_expect_tx(q_full(qs), Ly::kQStage);
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             if (lane == 1) {
               const int ks = jj % NK;
-              if (jj >= NK) ok = mbar_wait(k_empty(ks), ((jj / NK) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+              if (jj >= NK) ok = mbar_wait(k_empty(ks), ((jj / NK) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns);
               if (!ok) break;
               const uint32_t kdst = sbase + Ly::kOffK + ks * Ly::kKStage;
               mbar_expect_tx(k_full(ks), Ly::kKStage);
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
               tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full(ks), 128, T.g, row);
             } else {
               const int vs = jj % NV;
-              if (jj >= NV) ok = mbar_wait(v_empty(vs), ((jj / NV) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT);
+              if (jj >= NV) ok = mbar_wait(v_empty(vs), ((jj / NV) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns);
               if (!ok) break;
               const uint32_t vdst = sbase + Ly::kOffV + vs * Ly::kVStage;
               mbar_expect_tx(v_full(vs), Ly::kVStage);
@@ -356,10 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       bool pend_first = false;
       auto issue_pv = [&](int jp, bool first, int mtp) -> bool {
         const int b = jp & 1;
-        if (!mbar_wait(p_full(b), (jp >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        if (!mbar_wait(p_full(b), (jp >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns)) return false;
         const int vs = jp % NV;
-        if (!mbar_wait(v_full(vs), (jp / NV) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
-        if (first && mtp > 0 && !mbar_wait(o_empty, (mtp - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))
+        if (!mbar_wait(v_full(vs), (jp / NV) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns)) return false;
+        if (first && mtp > 0 && !mbar_wait(o_empty, (mtp - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))
           return false;
         tc_fence_after();
         const uint32_t vbase = sbase + Ly::kOffV + vs * Ly::kVStage;
@@ -376,14 +377,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         TileInfo T;
         if (!locate<KIND>(p, S, w, T)) break;
         const int qs = mt % NQ;
-        if (!(ok = mbar_wait(q_rot(qs), (mt / NQ) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+        if (!(ok = mbar_wait(q_rot(qs), (mt / NQ) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
         tc_fence_after();
         int j_lo, nkv;
         key_tiles<KIND>(p, T, &j_lo, &nkv);
         const uint32_t qbase = sbase + Ly::kOffQ + qs * Ly::kQStage;
         for (int j = 0; j < nkv; ++j) {
           const int ks = jj % NK;
-          if (!(ok = mbar_wait(k_full(ks), (jj / NK) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          if (!(ok = mbar_wait(k_full(ks), (jj / NK) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
           tc_fence_after();
           const int b = jj & 1;
           const uint32_t kbase = sbase + Ly::kOffK + ks * Ly::kKStage;
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // The four softmax warps take every decision together: a wait that fails in one
     // lane fails for the whole warp, so warp-collective tcgen05 ops never diverge.
     auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns));
     };
     int n_rot = 0;
     // Partial RoPE of M tile T in Q stage qs: the R x 32 cos/sin pairs are computed
@@ -450,15 +451,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       uint8_t* row = smem + Ly::kOffQ + qs * Ly::kQStage + m * 128;
       const int sw = m & 7;
       const float2* csr = cs + r * 32;
+      float amax = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         uint4* plo = reinterpret_cast<uint4*>(row + ((u ^ sw) << 4));
         uint4* phi = reinterpret_cast<uint4*>(row + (((u + 4) ^ sw) << 4));
         uint4 lo = *plo, hi = *phi;
-        rope_chunk_pair_cs(lo, hi, csr + 8 * u);
+        rope_chunk_pair_cs(lo, hi, csr + 8 * u, amax);
         *plo = lo;
         *phi = hi;
       }
+      if (amax > kF16Max && r < T.rows_valid) atomicOr(status, MIMO_STATUS_RANGE);
       fence_proxy_async_smem();
       mbar_arrive(q_rot(qs));
       return true;
@@ -721,8 +724,9 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
         if (!locate<0>(p, S, w, T)) break;
         const int row = T.krow_base + (T.qpos0 - 128 - T.kpos_base);
         if (lane == 0) {
+          if (p.withhold_q) break;  // failure-detection test: no query tile ever arrives
           const int b = mt & 1;
-          if (mt >= 2 && !(ok = mbar_wait(q_empty(b), ((mt >> 1) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)))
+          if (mt >= 2 && !(ok = mbar_wait(q_empty(b), ((mt >> 1) - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns)))
             break;
           const uint32_t qdst = sbase + Ly::kOffQ + b * Ly::kQStage;
           mbar_expect_tx(q_full(b), Ly::kQStage + Ly::kCSStage);
@@ -730,14 +734,14 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
             tma_load_3d(qdst + c * Ly::kQChunk, &p.tm_q, q_full(b), 64 * c, T.g * G, T.q_row0);
           tma_load_2d(sbase + Ly::kOffCS + b * Ly::kCSStage, &p.tm_cs, q_full(b), 0, T.q_row0);
         } else if (lane == 1) {
-          if (mt >= 1 && !(ok = mbar_wait(k_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          if (mt >= 1 && !(ok = mbar_wait(k_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
           const uint32_t kdst = sbase + Ly::kOffK;
           mbar_expect_tx(k_full, 3 * Ly::kKChunk);
           tma_load_3d(kdst, &p.tm_k0, k_full, 0, T.g, row);
           tma_load_3d(kdst + Ly::kKChunk, &p.tm_k12, k_full, 64, T.g, row);
           tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full, 128, T.g, row);
         } else {
-          if (mt >= 1 && !(ok = mbar_wait(v_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+          if (mt >= 1 && !(ok = mbar_wait(v_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
           const uint32_t vdst = sbase + Ly::kOffV;
           mbar_expect_tx(v_full, 2 * Ly::kVChunk);
           tma_load_3d(vdst, &p.tm_v, v_full, 0, T.g, row);
@@ -761,8 +765,8 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
       bool ok = true;
       auto issue_pv = [&](int t) -> bool {
         const int b = t & 1;
-        if (!mbar_wait(p_full(b), (t >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
-        if (!mbar_wait(v_full, t & 1, abort_flag, status, MIMO_STATUS_TIMEOUT)) return false;
+        if (!mbar_wait(p_full(b), (t >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns)) return false;
+        if (!mbar_wait(v_full, t & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns)) return false;
         tc_fence_after();
         const uint32_t reg = tmem + b * kSwaRegion;
 #pragma unroll
@@ -825,12 +829,12 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
         }
         if (progress) {
           t_last = global_timer_ns();
-        } else if (!*abort_flag && global_timer_ns() - t_last <= 2000000000ull) {
+        } else if (!*abort_flag && global_timer_ns() - t_last <= p.wait_ns) {
           __nanosleep(32);  // yield the issue slots this sub-partition shares with softmax warps
         } else if (*abort_flag) {
           ok = false;
           break;
-        } else if (global_timer_ns() - t_last > 2000000000ull) {
+        } else if (global_timer_ns() - t_last > p.wait_ns) {
           *abort_flag = 1;
           atomicOr(status, MIMO_STATUS_TIMEOUT);
           ok = false;
@@ -854,9 +858,10 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
       TileInfo T;
       if (!locate<0>(p, S, w, T)) break;
       const int b = mt & 1;
-      if (!(ok = mbar_wait(q_full(b), (mt >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT))) break;
+      if (!(ok = mbar_wait(q_full(b), (mt >> 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
       const float4* cs = reinterpret_cast<const float4*>(smem + Ly::kOffCS + b * Ly::kCSStage);
       uint8_t* qs = smem + Ly::kOffQ + b * Ly::kQStage;
+      float amax = 0.f;  // every row holds a real query (or TMA zero fill past total_q)
       // work item k: head h = k & 7, chunk pair u = (k >> 3) & 3, position r = k >> 5 (row 8r + h):
       // the 8 lanes of a shared-memory phase hit 8 distinct swizzled 16-byte groups of Q and
       // read one broadcast (cos, sin) address.
@@ -869,10 +874,11 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
         uint4* phi = reinterpret_cast<uint4*>(row + (((u + 4) ^ sw) << 4));
         uint4 lo = *plo, hi = *phi;
         // (cos, sin) of frequencies 8u..8u+7 at the row's position: 4 x float4
-        rope_chunk_pair_cs4(lo, hi, cs + (m / G) * 16 + 4 * u);
+        rope_chunk_pair_cs4(lo, hi, cs + (m / G) * 16 + 4 * u, amax);
         *plo = lo;
         *phi = hi;
       }
+      if (amax > kF16Max) atomicOr(status, MIMO_STATUS_RANGE);
       fence_proxy_async_smem();
       mbar_arrive(q_rot(b));
     }
@@ -885,7 +891,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
     const uint32_t t_lane = tmem + (uint32_t(quad * 32) << 16) + wg * kSwaRegion;
     const float c_log2 = p.scale_log2;
     auto wait_w = [&](uint32_t bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT));
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns));
     };
     for (int mt = wg, w = blockIdx.x + wg * gridDim.x;; mt += 2, w += 2 * gridDim.x) {
       TileInfo T;
@@ -1175,12 +1181,14 @@ __global__ void __launch_bounds__(256, 2) rope_k_contig_kernel(const RopeKParams
 #pragma unroll
     for (int i = 0; i < 8; ++i) rope_cos_sin(pos_k, p.rope.inv_freq[8 * u + i], &cs[i].x, &cs[i].y);
     uint4* dst = reinterpret_cast<uint4*>(p.ws_k + row * HKV * kRope) + u;
+    float amax = 0.f;
 #pragma unroll
     for (int g = 0; g < HKV; ++g) {
-      rope_chunk_pair_cs(a[g], b[g], cs);
+      rope_chunk_pair_cs(a[g], b[g], cs, amax);
       dst[g * (kRope / 8)] = a[g];
       dst[g * (kRope / 8) + 4] = b[g];
     }
+    if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
   }
   if (q_row) {
     const int pos_q = query_position(p, row);
@@ -1232,7 +1240,7 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
         for (int t = lane; t < kKRow; t += 32) kd[t] = make_uint4(0, 0, 0, 0);
         for (int t = lane; t < kVRow; t += 32) vd[t] = make_uint4(0, 0, 0, 0);
       } else {
-        const long entry = long(s) * kPage + (pos % kPage);
+        const long entry = long(s) * p.ring_slots + (pos % p.ring_slots);
         const uint4* ks = reinterpret_cast<const uint4*>(p.ring_k + entry * HKV * kDqk);
         const uint4* vs = reinterpret_cast<const uint4*>(p.ring_v + entry * HKV * kDv);
         uint4 kr[(kKRow + 31) / 32], vr[(kVRow + 31) / 32];
@@ -1279,7 +1287,9 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
         cs[f].y = __shfl_sync(0xffffffffu, s_j, 8 * pu + f);
       }
       if (has_pair) {
-        rope_chunk_pair_cs(ra, rb, cs);
+        float amax = 0.f;
+        rope_chunk_pair_cs(ra, rb, cs, amax);
+        if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
         kd[pg * (kDqk / 8) + pu] = ra;
         kd[pg * (kDqk / 8) + pu + 4] = rb;
       }

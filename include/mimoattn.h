@@ -57,6 +57,9 @@ extern "C" {
 /* Device status bits reported by mimo_status_poll(). */
 #define MIMO_STATUS_TIMEOUT 1u    /* a bounded barrier / copy wait ran out */
 #define MIMO_STATUS_BAD_INDEX 2u  /* a page id, slot or position outside its cache */
+#define MIMO_STATUS_RANGE 4u      /* a rotated query / key component beyond fp16's range,
+                                     stored saturated at +-65504 */
+#define MIMO_STATUS_BAD_SCALE 8u  /* an E4M3 dequantisation scale not finite and positive */
 
 /* The attention layer.  num_q_heads 64, head_dim_qk 192, head_dim_v 128 and
  * rope_dim 64 are required; num_kv_heads is 8 or 4. */
@@ -87,9 +90,26 @@ typedef struct {
  * device and launches nothing. */
 MIMO_API int mimo_window_from_left_right(int left, int right, int* window);
 
+/* KV cache layouts.  The serving pages keep window-sized KV for the sliding-window
+ * layers and paged KV in blocks of 128 positions for the global layers (gaudi-cookbook
+ * "MiMo-V2.6-Flash-RL", section "Launch": MIMO_SWA_KV_GROUPS=1 gives the 39 sliding
+ * layers window-sized KV, --block-size 128), and their exact decode window keeps one
+ * block more than the window with the oldest block masked (same page, "Fixes" table,
+ * swa-decode-window).
+ *   MIMO_CACHE_PAGED: [num_pages, 128, Hkv, D]; position p of sequence s sits in page
+ *     block_table[s][p / 128], slot p % 128.
+ *   MIMO_CACHE_RING: [num_seqs, ring_slots, Hkv, D]; position p of sequence s sits in slot
+ *     p % ring_slots, so the ring holds the last ring_slots positions appended.  ring_slots
+ *     (a field of the prefill, decode and append arguments; 0 means 128) is a multiple of
+ *     16 in 128..512.  The model's window of 128 keys fits 128 slots.  The SGLang window of
+ *     the query plus 128 previous keys (radixark miles docs "MiMo-V2.6-Flash", section 5.4)
+ *     needs at least 129 slots to decode, because appending the query's own key overwrites
+ *     the oldest slot: 144 is the smallest ring that serves it. */
 #define MIMO_CACHE_NONE 0
-#define MIMO_CACHE_PAGED 1 /* [num_pages, 128, Hkv, D] pages of 128 positions, via block_table */
-#define MIMO_CACHE_RING 2  /* [num_seqs, 128, Hkv, D]: position p of sequence s in slot p % 128 */
+#define MIMO_CACHE_PAGED 1
+#define MIMO_CACHE_RING 2
+#define MIMO_RING_SLOTS_DEFAULT 128
+#define MIMO_RING_SLOTS_MAX 512
 
 /* Cache element formats (mimo_decode_args.cache_dtype, mimo_append_args.cache_dtype).
  *   MIMO_DTYPE_BF16: key dims 0..63 (the rotated part) as IEEE fp16, key dims
@@ -116,9 +136,10 @@ MIMO_API int mimo_window_from_left_right(int left, int right, int* window);
  * are read from the cache, where keys are stored already rotated.
  *
  *   MIMO_CACHE_NONE : all keys are new; k, v, cu_seqlens_k required.
- *   MIMO_CACHE_RING : sliding-window chunk: the ring holds the positions
- *                     cache_lens[s]-128 .. cache_lens[s]-1 (the prefix tail, not yet
- *                     overwritten by this chunk); requires window in 1..129.
+ *   MIMO_CACHE_RING : sliding-window chunk: the ring holds the prefix tail, positions
+ *                     cache_lens[s]-ring_slots .. cache_lens[s]-1 (not yet overwritten by
+ *                     this chunk), of which the last 128 are read; requires window in
+ *                     1..129 (a window reaches at most 128 positions before the chunk).
  *   MIMO_CACHE_PAGED: all keys come from the paged cache (append the chunk with
  *                     mimo_kv_append first); k, v, cu_seqlens_k must be NULL and
  *                     cache_lens[s] is the full context length.
@@ -159,6 +180,7 @@ typedef struct {
    * cudaEventElapsedTime gives that kernel's device time. */
   void* ev_kernel_begin;
   void* ev_kernel_end;
+  int ring_slots; /* MIMO_CACHE_RING: slots per sequence of the ring (0 = 128) */
 } mimo_prefill_args;
 
 /* Bytes of workspace mimo_attn_prefill needs for these sizes. */
@@ -168,10 +190,25 @@ MIMO_API size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_q, int 
 MIMO_API int mimo_attn_prefill(const mimo_prefill_args* args, void* stream);
 
 /*
+ * Failure-detection test of the prefill (no counterpart in the pages: it exercises this
+ * library's own bounded waits).  Validates and enqueues exactly what mimo_attn_prefill
+ * would, except that the attention kernel's producer never loads a query tile, so the
+ * roles waiting for one give up after wait_limit_ns (1e6..1e10 ns), set
+ * MIMO_STATUS_TIMEOUT in the device status word, wait for their copies and tensor-core
+ * operations already in flight, free their tensor memory and return; the outputs are
+ * left unspecified.  mimo_status_poll() then returns MIMO_ERR_TIMEOUT, and later calls
+ * run normally.  Nothing faults and nothing waits without a limit.
+ */
+MIMO_API int mimo_attn_prefill_stall_test(const mimo_prefill_args* args, void* stream,
+                                          unsigned long long wait_limit_ns);
+
+/*
  * Decode: one query token per sequence.  Token s sits at position
  * seq_lens[s] - 1 and the cache already holds positions 0 .. seq_lens[s]-1
  * (append the token with mimo_kv_append first).  Sliding-window layers use a
- * ring cache (only the last 128 positions are kept); global layers a paged cache.
+ * ring cache (the last ring_slots positions are kept; window in 1..ring_slots),
+ * global layers a paged cache (gaudi-cookbook "MiMo-V2.6-Flash-RL", "Launch":
+ * window-sized KV for the sliding layers, blocks of 128 positions).
  *
  * Layouts: q [batch, 64, 192] bf16 pre-RoPE; out [batch, 64, 128] bf16;
  * lse [batch, 64] fp32 or NULL.  max_seq_len is a host-side upper bound of
@@ -202,6 +239,7 @@ typedef struct {
   int cache_dtype;          /* MIMO_DTYPE_BF16 (default 0) or MIMO_DTYPE_FP8_E4M3 */
   const float* k_dequant;   /* FP8: device fp32 [num_kv_heads] key scales, else NULL */
   const float* v_dequant;   /* FP8: device fp32 [num_kv_heads] value scales, else NULL */
+  int ring_slots;           /* MIMO_CACHE_RING: slots per sequence of the ring (0 = 128) */
 } mimo_decode_args;
 
 /* Bytes of workspace mimo_attn_decode needs (split-KV partials). */
@@ -223,7 +261,8 @@ MIMO_API int mimo_attn_decode(const mimo_decode_args* args, void* stream);
  *   - Nothing is allocated: no cudaMalloc / cudaFree, no allocating library call.
  *   - The first call on each device looks up that device's copy of the array
  *     (cudaGetSymbolAddress, with the device current): make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is looked up again when the
+ *     device's context has changed since (after a device reset).
  *   - Problems whose partials need more than MIMO_DECODE_NOALLOC_MAX_BYTES
  *     (mimo_attn_decode_workspace_size of the same sizes) are rejected with
  *     MIMO_ERR_WORKSPACE before anything is enqueued.
@@ -238,11 +277,17 @@ MIMO_API int mimo_attn_decode_noalloc(const mimo_decode_args* args, void* stream
 /*
  * KV append: rotates the first 64 dims of each new key at its position (the
  * layer's RoPE base, angles from float64) and stores key and value (value
- * unscaled) in the cache: ring slot pos % 128 of sequence seq_idx[t], or page
- * block_table[seq_idx[t]][pos / 128], slot pos % 128.
+ * unscaled) in the cache: ring slot pos % ring_slots of sequence seq_idx[t], or page
+ * block_table[seq_idx[t]][pos / 128], slot pos % 128 (the cache layouts above:
+ * gaudi-cookbook "MiMo-V2.6-Flash-RL", "Launch").
  *
  * Layouts: k_new [num_tokens, Hkv, 192] bf16 pre-RoPE; v_new [num_tokens, Hkv, 128];
  * pos, seq_idx: device int32 [num_tokens].  Two tokens must not target the same slot.
+ * A token whose sequence, position or page lies outside the cache is skipped and sets
+ * MIMO_STATUS_BAD_INDEX.  For an E4M3 cache every k_dequant / v_dequant scale must be
+ * finite and positive; a token of a KV head whose scale is not is skipped and sets
+ * MIMO_STATUS_BAD_SCALE.  A rotated key component beyond the fp16 range (|x| > 65504)
+ * is stored as +-65504 and sets MIMO_STATUS_RANGE (bf16 caches).
  */
 typedef struct {
   int num_tokens;
@@ -265,6 +310,7 @@ typedef struct {
   int cache_dtype;          /* MIMO_DTYPE_BF16 (default 0) or MIMO_DTYPE_FP8_E4M3 */
   const float* k_dequant;   /* FP8: device fp32 [num_kv_heads], else NULL */
   const float* v_dequant;
+  int ring_slots;           /* MIMO_CACHE_RING: slots per sequence of the ring (0 = 128) */
 } mimo_append_args;
 
 MIMO_API int mimo_kv_append(const mimo_append_args* args, void* stream);

@@ -72,7 +72,23 @@ int main(void) {
     d.layer.window = 0;
     d.batch = 0; /* an empty batch is a no-op */
     CHECK(mimo_attn_decode(&d, NULL) == MIMO_OK);
+    d.ring_slots = 136; /* not a multiple of the 16-key tile */
+    d.batch = 1;
+    d.max_seq_len = 16;
+    d.cache_kind = MIMO_CACHE_RING;
+    CHECK(mimo_attn_decode(&d, NULL) == MIMO_ERR_INVALID_ARG);
+    CHECK(strstr(mimo_last_error(), "ring_slots") != NULL);
   }
+  {
+    mimo_prefill_args a;
+    memset(&a, 0, sizeof(a));
+    a.layer = model_layer(8);
+    /* the stall test checks its wait limit before anything else */
+    CHECK(mimo_attn_prefill_stall_test(&a, NULL, 10ull) == MIMO_ERR_INVALID_ARG);
+  }
+  CHECK(MIMO_STATUS_TIMEOUT == 1u && MIMO_STATUS_BAD_INDEX == 2u && MIMO_STATUS_RANGE == 4u &&
+        MIMO_STATUS_BAD_SCALE == 8u);
+  CHECK(MIMO_RING_SLOTS_DEFAULT == 128 && MIMO_RING_SLOTS_MAX == 512);
   printf("ok\n");
   return 0;
 }

@@ -107,6 +107,11 @@ def _prefill_args(**over):
     ({"cache_kind": M.MIMO_CACHE_PAGED}, M.MIMO_ERR_INVALID_ARG),          # paged: k/v must be NULL
     ({"cache_kind": M.MIMO_CACHE_RING, "layer.window": 0}, M.MIMO_ERR_INVALID_ARG),
     ({"layer.sink": C.c_void_p(FAKE + 2)}, M.MIMO_ERR_INVALID_ARG),
+    ({"ring_slots": 96}, M.MIMO_ERR_INVALID_ARG),                          # below 128
+    ({"ring_slots": 136}, M.MIMO_ERR_INVALID_ARG),                         # not a multiple of 16
+    ({"ring_slots": 528}, M.MIMO_ERR_INVALID_ARG),                         # above 512
+    ({"cache_kind": M.MIMO_CACHE_RING, "layer.window": 130, "k_cache": C.c_void_p(FAKE),
+      "v_cache": C.c_void_p(FAKE), "cache_lens": C.c_void_p(FAKE)}, M.MIMO_ERR_INVALID_ARG),
 ])
 def test_prefill_validation(over, code):
     a = _prefill_args(**over)
@@ -151,6 +156,10 @@ def _decode_args(**over):
     ({"cache_dtype": M.MIMO_DTYPE_FP8_E4M3}, M.MIMO_ERR_INVALID_ARG),     # E4M3 needs dequant scales
     ({"cache_dtype": M.MIMO_DTYPE_FP8_E4M3, "k_dequant": C.c_void_p(FAKE), "v_dequant": C.c_void_p(FAKE + 2)},
      M.MIMO_ERR_INVALID_ARG),                                             # misaligned scales
+    ({"cache_kind": M.MIMO_CACHE_RING, "layer.window": 129}, M.MIMO_ERR_INVALID_ARG),   # 128 slots < 129 keys
+    ({"cache_kind": M.MIMO_CACHE_RING, "layer.window": 145, "ring_slots": 144}, M.MIMO_ERR_INVALID_ARG),
+    ({"ring_slots": 100}, M.MIMO_ERR_INVALID_ARG),
+    ({"ring_slots": 1024}, M.MIMO_ERR_INVALID_ARG),
 ])
 def test_decode_validation(over, code):
     a = _decode_args(**over)
@@ -169,6 +178,29 @@ def test_append_validation():
     assert M.lib().mimo_kv_append(C.byref(a), None) == M.MIMO_ERR_UNSUPPORTED
     a.rope_dim, a.num_tokens = 64, 0
     assert M.lib().mimo_kv_append(C.byref(a), None) == M.MIMO_OK                 # nothing to append
+
+
+def test_ring_slots_constants_match_header():
+    src = open(HEADER).read()
+    for name in ["MIMO_RING_SLOTS_DEFAULT", "MIMO_RING_SLOTS_MAX", "MIMO_STATUS_TIMEOUT", "MIMO_STATUS_BAD_INDEX",
+                 "MIMO_STATUS_RANGE", "MIMO_STATUS_BAD_SCALE"]:
+        m = re.search(rf"#define {name} (\d+)", src)
+        assert m and int(m.group(1)) == getattr(M, name), name
+
+
+@pytest.mark.parametrize("ns", [0, 999_999, 10_000_000_001])
+def test_stall_test_rejects_limits_outside_its_range(ns):
+    a = _prefill_args()
+    assert M.lib().mimo_attn_prefill_stall_test(C.byref(a), None, ns) == M.MIMO_ERR_INVALID_ARG
+    assert M.lib().mimo_last_error().startswith(b"mimo_attn_prefill_stall_test")
+
+
+def test_append_rejects_bad_ring_slots():
+    a = M.MimoAppendArgs()
+    a.num_tokens, a.num_kv_heads, a.head_dim_qk, a.head_dim_v, a.rope_dim, a.rope_base = 4, 8, 192, 128, 64, 1e4
+    a.k_new = a.v_new = a.pos = a.seq_idx = a.k_cache = a.v_cache = C.c_void_p(FAKE)
+    a.cache_kind, a.num_seqs, a.ring_slots = M.MIMO_CACHE_RING, 1, 200
+    assert M.lib().mimo_kv_append(C.byref(a), None) == M.MIMO_ERR_INVALID_ARG
 
 
 def test_status_poll_rejects_null():

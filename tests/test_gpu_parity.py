@@ -12,7 +12,8 @@ import pytest
 import oracle
 from workloads import configs, synth
 
-from .util import (chunked_cfg, decode_cfg, dev_bf16, dev_f32, dev_i32, host_f64, parity, prefill_cfg)
+from .util import (check_prefill, chunked_cfg, decode_cfg, dev_bf16, dev_f32, dev_i32, host_f64, make_prefill, parity,
+                   prefill_cfg)
 
 pytestmark = pytest.mark.gpu
 
@@ -25,45 +26,26 @@ def _gpu(cuda_ok):
     assert M.status_poll() == 0, "device status word reported a timeout or a bad index"
 
 
-def make_prefill(lens, hkv, base, window, sink, seed, klens=None):
-    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    klens = lens if klens is None else klens
-    cuk = np.concatenate([[0], np.cumsum(klens)]).astype(np.int32)
-    q = configs.bf16_normal(seed, 1, (int(cu[-1]), 64, 192))
-    k = configs.bf16_normal(seed, 2, (int(cuk[-1]), hkv, 192))
-    v = configs.bf16_normal(seed, 3, (int(cuk[-1]), hkv, 128))
-    s = synth.normal_f32(synth.stream_seed(seed, 4), (64,)) if sink else None
-    return configs.Prefill(configs.Layer("swa" if window else "global", hkv, base, window, s), q, k, v, cu, cuk)
-
-
-def check_prefill(cfg, rows=None, what=""):
-    out, lse = prefill_cfg(cfg)
-    ro, rl = oracle.prefill(cfg, rows=rows)
-    if rows is not None:
-        import torch
-        idx = torch.as_tensor(np.asarray(rows), dtype=torch.long, device=out.device)
-        out, lse = out[idx], lse[idx]
-    return parity(out, lse, ro, rl, what)
-
-
 # ----------------------------------------------------------------------------- KV append
 
-@pytest.mark.parametrize("kind", ["ring", "paged"])
+@pytest.mark.parametrize("kind", ["ring", "ring144", "paged"])
 def test_kv_append(kind):
     import torch
     import global_attention_attn_b200 as M
-    # at most 128 tokens per sequence for the ring: two tokens of one call must not share a slot
-    n, hkv, base = (300, 8, 1e4) if kind == "ring" else (700, 4, 1e7)
+    # at most `slots` tokens per sequence for a ring: two tokens of one call must not share a slot
+    slots = 144 if kind == "ring144" else 128
+    n, hkv, base = (3 * slots, 8, 1e4) if kind.startswith("ring") else (700, 4, 1e7)
     k = configs.bf16_normal(41, 1, (n, hkv, 192))
     v = configs.bf16_normal(41, 2, (n, hkv, 128))
     seq = (np.arange(n) % 3).astype(np.int32)
     pos = (np.arange(n) // 3 + np.array([0, 5, 120000])[seq]).astype(np.int32)
-    if kind == "ring":
-        kc = torch.zeros((3, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
-        vc = torch.zeros((3, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
+    if kind.startswith("ring"):
+        kc = torch.zeros((3, slots, hkv, 192), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros((3, slots, hkv, 128), dtype=torch.bfloat16, device="cuda")
         M.mimo_kv_append(dev_bf16(k), dev_bf16(v), dev_i32(pos), dev_i32(seq), rope_base=base,
-                         cache_kind=M.MIMO_CACHE_RING, k_cache=kc, v_cache=vc, num_seqs=3)
-        where = {(int(seq[t]), int(pos[t] % 128)): t for t in range(n)}
+                         cache_kind=M.MIMO_CACHE_RING, k_cache=kc, v_cache=vc, num_seqs=3,
+                         ring_slots=0 if slots == 128 else slots)
+        where = {(int(seq[t]), int(pos[t] % slots)): t for t in range(n)}
     else:
         maxp = (int(pos.max()) // 128) + 1
         bt = (synth.permutation(7, 3 * maxp).reshape(3, maxp)).astype(np.int32)
@@ -233,14 +215,34 @@ def test_decode_fp8_split_boundaries_and_window():
 
 
 def test_decode_fp8_b64_full_scale():
-    """64 sequences, contexts U[4096, 65536] over an E4M3 paged cache, checked on 8 sequences."""
-    import torch
+    """64 sequences, contexts U[4096, 65536] over an E4M3 paged cache, every sequence checked."""
     cfg = configs.decode_fp8()
     out, lse = decode_cfg(cfg)
-    seqs = np.array(sorted(set([0, 63] + list(synth.permutation(79, 64)[:6]))))
-    ro, rl = oracle.decode(cfg, seqs=seqs)
-    idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "fp8 64-sequence decode scale, sampled sequences")
+    ro, rl = oracle.decode(cfg)
+    parity(out, lse, ro, rl, "fp8 64-sequence decode, all sequences")
+
+
+@pytest.mark.parametrize("ring_slots,window", [(144, 129), (144, 128), (256, 129), (512, 300), (128, 5)])
+def test_decode_ring_slots(ring_slots, window):
+    """Rings longer than 128 slots: the SGLang window of the query plus 128 previous keys
+    (radixark miles docs "MiMo-V2.6-Flash", section 5.4) decoded from a ring that keeps one
+    16-key tile more than the window (144 slots), and wider rings and windows."""
+    import dataclasses
+    sw, _ = configs.decode_batch(seed=330 + ring_slots + window, B=12, ctx_range=(1, 2000), ring_slots=ring_slots)
+    sw.layer = dataclasses.replace(sw.layer, window=window)
+    sw.ctx[:3] = [1, window - 1, window]
+    out, lse = decode_cfg(sw)
+    parity(out, lse, *oracle.decode(sw), f"ring {ring_slots} decode, window {window}")
+
+
+def test_decode_ring_rejects_a_window_beyond_its_slots():
+    import global_attention_attn_b200 as M
+    sw, _ = configs.decode_batch(seed=340, B=2, ctx_range=(200, 300))
+    import dataclasses
+    sw.layer = dataclasses.replace(sw.layer, window=129)
+    with pytest.raises(M.MimoError) as e:
+        decode_cfg(sw)
+    assert e.value.code == M.MIMO_ERR_INVALID_ARG
 
 
 @pytest.fixture(scope="module")
@@ -258,11 +260,8 @@ def test_decode_b64_swa_ring(dec64):
 def test_decode_b64_global_paged(dec64):
     _, gl = dec64
     out, lse = decode_cfg(gl)
-    seqs = np.array(sorted(set([0, 63] + list(synth.permutation(77, 64)[:6]))))
-    ro, rl = oracle.decode(gl, seqs=seqs)
-    import torch
-    idx = torch.as_tensor(seqs, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "decode b64 global paged, sampled sequences")
+    ro, rl = oracle.decode(gl)
+    parity(out, lse, ro, rl, "decode b64 global paged, all 64 sequences")
 
 
 # ----------------------------------------------------------------------------- prefill: sliding window
@@ -333,8 +332,9 @@ def test_prefill_global_with_sink_and_wide_window():
 
 def test_prefill_global_s16384_sampled():
     cfg = configs.global_causal_prefill()
-    rows = configs.sample_rows(22, 16384, 96, always=(0, 1, 7, 8, 127, 128, 129, 8191, 16383))
-    check_prefill(cfg, rows=rows, what="global prefill s16384 (sampled rows)")
+    rows = configs.sample_rows(22, 16384, 1024, always=(0, 1, 7, 8, 127, 128, 129, 8191, 16383))
+    assert len(rows) == 1024
+    check_prefill(cfg, rows=rows, what="global prefill s16384 (1024 sampled rows)")
 
 
 # ----------------------------------------------------------------------------- chunked prefill
@@ -364,6 +364,15 @@ def test_chunked_swa_window_left_right_128_0():
     parity(out, lse, ro, rl, swa.name)
 
 
+def test_chunked_swa_from_a_256_slot_ring_window_129():
+    """The sliding-window chunk reads its 128 halo positions from a ring longer than 128."""
+    import dataclasses
+    _, swa = configs.chunked_prefill(seed=57, prefix=1000, chunk=300, n_sample=300, ring_slots=256)
+    swa.layer = dataclasses.replace(swa.layer, window=129)
+    out, lse = chunked_cfg(swa)
+    parity(out, lse, *oracle.chunked(swa, rows=np.arange(300)), "swa chunk from a 256-slot ring, window 129")
+
+
 def test_chunked_8192_on_120832():
     glb, swa = configs.chunked_prefill()
     out, lse = chunked_cfg(swa)
@@ -372,10 +381,12 @@ def test_chunked_8192_on_120832():
     idx = torch.as_tensor(swa.sample_rows, dtype=torch.long, device=out.device)
     parity(out[idx], lse[idx], ro, rl, "swa chunk 8192 on 120832 (1024 sampled rows)")
     out, lse = chunked_cfg(glb)
-    rows = configs.sample_rows(4, 8192, 48, always=(0, 126, 127, 128, 8191))
+    # the 1024 seeded rows of the workload (rows 0, 126, 127, 128 and 8191 among them)
+    rows = glb.sample_rows
+    assert len(rows) == 1024 and {0, 126, 127, 128, 8191} <= set(int(r) for r in rows)
     ro, rl = oracle.chunked(glb, rows=rows)
     idx = torch.as_tensor(rows, dtype=torch.long, device=out.device)
-    parity(out[idx], lse[idx], ro, rl, "global chunk 8192 on 120832 (sampled rows)")
+    parity(out[idx], lse[idx], ro, rl, "global chunk 8192 on 120832 (1024 sampled rows)")
 
 
 # ----------------------------------------------------------------------------- cross-path
@@ -436,35 +447,32 @@ def test_verify_draft_tokens(q_len):
 
 def test_verify_b64_full_scale(dec64):
     """Verification at the decode workload's scale (64 sequences, contexts up to 64K) on the
-    64-sequence decode caches, checked on the rows of 4 sampled sequences."""
-    import torch
+    64-sequence decode caches, every draft row of every sequence checked."""
     _, gl = dec64
     glb, swa = configs.verify(B=64, q_len=4, decode=gl)
-    seqs = np.array([0, 17, 42, 63])
-    rows = (seqs[:, None] * 4 + np.arange(4)[None, :]).reshape(-1)
     for cfg in (glb, swa):
         out, lse = chunked_cfg(cfg)
-        ro, rl = oracle.chunked(cfg, rows=rows)
-        idx = torch.as_tensor(rows, dtype=torch.long, device=out.device)
-        parity(out[idx], lse[idx], ro, rl, cfg.name)
+        ro, rl = oracle.chunked(cfg, rows=np.arange(64 * 4))
+        parity(out, lse, ro, rl, cfg.name)
 
 
 def test_decode_matches_last_prefill_row():
     """Appending a sequence to the caches and decoding its last token gives the last prefill row."""
     import torch
     import global_attention_attn_b200 as M
-    for hkv, base, window, sink in [(8, 1e4, 128, True), (4, 1e7, 0, False)]:
+    for hkv, base, window, sink, slots in [(8, 1e4, 128, True, 128), (8, 1e4, 129, True, 144),
+                                           (4, 1e7, 0, False, 0)]:
         S = 700
-        cfg = make_prefill([S], hkv, base, window, sink, 500 + hkv)
+        cfg = make_prefill([S], hkv, base, window, sink, 500 + hkv + window)
         out, lse = prefill_cfg(cfg)
-        # the ring keeps the last 128 positions: append only those (one call may not reuse a slot)
-        first = S - 128 if window else 0
+        # the ring keeps the last `slots` positions: append only those (one call may not reuse a slot)
+        first = S - slots if window else 0
         pos = np.arange(first, S, dtype=np.int32)
         seq = np.zeros(S - first, np.int32)
         if window:
-            kc = torch.zeros((1, 128, hkv, 192), dtype=torch.bfloat16, device="cuda")
-            vc = torch.zeros((1, 128, hkv, 128), dtype=torch.bfloat16, device="cuda")
-            extra = dict(cache_kind=M.MIMO_CACHE_RING)
+            kc = torch.zeros((1, slots, hkv, 192), dtype=torch.bfloat16, device="cuda")
+            vc = torch.zeros((1, slots, hkv, 128), dtype=torch.bfloat16, device="cuda")
+            extra = dict(cache_kind=M.MIMO_CACHE_RING, ring_slots=slots)
         else:
             npg = (S + 127) // 128
             bt = dev_i32(synth.permutation(3, npg)[None, :])

@@ -153,3 +153,56 @@ def test_cp_rejects_windows_beyond_the_halo():
     for w in (0, 130):
         with pytest.raises(ValueError):
             cp.prefill_with_halo(q, None, None, [4], [0], None, None, rope_base=1e4, window=w)
+
+
+def _cp_stream_worker(rank, world, port):
+    """With a caller stream, every step of the context-parallel prefill (the ring appends,
+    the NCCL transfers, the prefill) runs while that stream is the current one, because
+    torch.distributed orders its transfers against the current stream."""
+    _init(rank, world, port)
+    from global_attention_attn_b200 import cp
+    state = {"inside": False, "calls": []}
+
+    class Scope:
+        def __init__(self, s):
+            assert s == "caller-stream"
+
+        def __enter__(self):
+            state["inside"] = True
+
+        def __exit__(self, *a):
+            state["inside"] = False
+
+    saved = (torch.cuda.stream, cp.fill_ring_tail, cp.exchange_halo, cp.prefill_with_halo)
+    try:
+        torch.cuda.stream = Scope
+
+        def fake_fill(rk, rv, k, v, chunk_lens, start_pos, *, rope_base, stream=None):
+            state["calls"].append(("append", state["inside"], stream))
+
+        def rec_exchange(*a, **kw):
+            state["calls"].append(("exchange", state["inside"], None))
+            return saved[2](*a, **kw)
+
+        def fake_prefill(*a, stream=None, **kw):
+            state["calls"].append(("prefill", state["inside"], stream))
+            return "out", "lse"
+
+        cp.fill_ring_tail, cp.exchange_halo, cp.prefill_with_halo = fake_fill, rec_exchange, fake_prefill
+        q = torch.zeros((300, 64, 192), dtype=torch.bfloat16)
+        k = torch.zeros((300, 2, 192), dtype=torch.bfloat16)
+        res = cp.swa_prefill_context_parallel(q, k, k, [300], [300 * rank], rope_base=1e4, window=128,
+                                              stream="caller-stream")
+        assert res == ("out", "lse")
+        names = [c[0] for c in state["calls"]]
+        assert names == (["exchange", "append", "prefill"] if rank + 1 < world else ["exchange", "prefill"]), names
+        # inside the caller's stream scope, with no other stream handed down
+        assert all(inside and s is None for _, inside, s in state["calls"]), state["calls"]
+        assert not state["inside"]
+    finally:
+        torch.cuda.stream, cp.fill_ring_tail, cp.exchange_halo, cp.prefill_with_halo = saved
+        dist.destroy_process_group()
+
+
+def test_cp_runs_every_step_on_the_caller_stream():
+    _run(_cp_stream_worker, 2)

@@ -14,7 +14,7 @@ import pytest
 import global_attention_attn_b200 as M
 from workloads import configs
 
-from .util import LSE_MAX_ABS, O_MAX_ABS, O_MEAN_ABS, dev_bf16, dev_f32, dev_i32
+from .util import LSE_MAX_ABS, O_MAX_ABS, O_MEAN_ABS, dev_bf16, dev_f32, dev_i32, dev_u8, parity
 
 
 def test_noalloc_rejects_oversize_before_touching_the_device():
@@ -29,27 +29,38 @@ def test_noalloc_rejects_oversize_before_touching_the_device():
     assert b"static scratch" in M.lib().mimo_last_error()
 
 
-def _case(seed, B, ctx_range):
-    _, gl = configs.decode_batch(seed=seed, B=B, ctx_range=ctx_range)
+def _case(seed, B, ctx_range, fp8=False):
+    if fp8:
+        gl = configs.decode_fp8(seed=seed, B=B, ctx_range=ctx_range)
+        kc, vc = dev_u8(gl.k_cache), dev_u8(gl.v_cache)
+        extra = dict(cache_dtype=M.MIMO_DTYPE_FP8_E4M3, k_dequant=dev_f32(gl.k_dequant),
+                     v_dequant=dev_f32(gl.v_dequant))
+    else:
+        _, gl = configs.decode_batch(seed=seed, B=B, ctx_range=ctx_range)
+        kc, vc = dev_bf16(gl.k_cache), dev_bf16(gl.v_cache)
+        extra = {}
     L = gl.layer
-    t = dict(q=dev_bf16(gl.q), ctx=dev_i32(gl.ctx), kc=dev_bf16(gl.k_cache), vc=dev_bf16(gl.v_cache),
-             bt=dev_i32(gl.block_table), pool=gl.k_cache.shape[0], max_len=int(gl.ctx.max()), L=L)
-    return t
+    return dict(cfg=gl, q=dev_bf16(gl.q), ctx=dev_i32(gl.ctx), kc=kc, vc=vc, bt=dev_i32(gl.block_table),
+                pool=gl.k_cache.shape[0], max_len=int(gl.ctx.max()), L=L, extra=extra)
 
 
 def _kw(t):
     return dict(max_seq_len=t["max_len"], num_kv_heads=t["L"].num_kv_heads, rope_base=t["L"].rope_base,
                 window=t["L"].window, cache_kind=M.MIMO_CACHE_PAGED, k_cache=t["kc"], v_cache=t["vc"],
-                block_table=t["bt"], num_pages=t["pool"], sink=dev_f32(t["L"].sink))
+                block_table=t["bt"], num_pages=t["pool"], sink=dev_f32(t["L"].sink), **t["extra"])
 
 
 @pytest.mark.gpu
 def test_noalloc_decode_matches_decode_on_two_calls(cuda_ok):
+    """Two calls in a row with different sizes and cache formats (bf16, then E4M3): the
+    second finds the first call's partials in the shared scratch and must not depend on
+    them.  Each output equals mimo_attn_decode's with a caller workspace and the oracle's,
+    and no device memory is taken: neither torch's allocator nor the device's free memory
+    (which also sees a cudaMalloc inside the library) changes across a call."""
     import torch
+    import oracle
     M.lib()
-    # two calls in a row with different sizes: the second finds the first call's partials in
-    # the shared scratch and must not depend on them
-    cases = [_case(901, 8, (2000, 3000)), _case(902, 5, (700, 1500))]
+    cases = [_case(901, 8, (2000, 3000)), _case(902, 5, (700, 1500), fp8=True)]
     for t in cases:
         assert 0 < M.decode_workspace_size(t["q"].shape[0], t["max_len"], 4, 0) <= M.DECODE_NOALLOC_MAX_BYTES
     refs = [M.mimo_attn_decode(t["q"], t["ctx"], **_kw(t)) for t in cases]
@@ -58,13 +69,16 @@ def test_noalloc_decode_matches_decode_on_two_calls(cuda_ok):
         B = t["q"].shape[0]
         out = torch.empty((B, 64, 128), dtype=torch.bfloat16, device="cuda")
         lse = torch.empty((B, 64), dtype=torch.float32, device="cuda")
-        before = torch.cuda.memory_allocated()
+        torch.cuda.synchronize()
+        before, free_before = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         M.mimo_attn_decode_noalloc(t["q"], t["ctx"], out=out, lse=lse, **_kw(t))
+        torch.cuda.synchronize()
         assert torch.cuda.memory_allocated() == before
+        assert torch.cuda.mem_get_info()[0] == free_before
         outs.append((out, lse))
-    torch.cuda.synchronize()
-    for (ro, rl), (o, l) in zip(refs, outs):
+    for t, (ro, rl), (o, l) in zip(cases, refs, outs):
         d = (o.float() - ro.float()).abs()
         assert d.max().item() <= O_MAX_ABS and d.mean().item() <= O_MEAN_ABS
         assert (l - rl).abs().max().item() <= LSE_MAX_ABS
+        parity(o, l, *oracle.decode(t["cfg"]), "no-alloc decode against the oracle")
     assert M.status_poll() == 0

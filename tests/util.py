@@ -69,7 +69,7 @@ def decode_cfg(cfg, **kw):
         extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
                      num_pages=cfg.k_cache.shape[0])
     else:
-        extra = dict(cache_kind=M.MIMO_CACHE_RING)
+        extra = dict(cache_kind=M.MIMO_CACHE_RING, ring_slots=cfg.k_cache.shape[1])
     if cfg.cache_dtype == M.MIMO_DTYPE_FP8_E4M3:
         kc, vc = dev_u8(cfg.k_cache), dev_u8(cfg.v_cache)
         extra.update(cache_dtype=cfg.cache_dtype, k_dequant=dev_f32(cfg.k_dequant), v_dequant=dev_f32(cfg.v_dequant))
@@ -107,4 +107,31 @@ def chunked_cfg(cfg):
     return M.mimo_attn_prefill(q, dev_bf16(cfg.k_new), dev_bf16(cfg.v_new), cu, cu, num_kv_heads=L.num_kv_heads,
                                rope_base=L.rope_base, window=L.window, sink=dev_f32(L.sink),
                                cache_lens=dev_i32(cfg.start), cache_kind=M.MIMO_CACHE_RING,
-                               k_cache=dev_bf16(cfg.k_cache), v_cache=dev_bf16(cfg.v_cache))
+                               k_cache=dev_bf16(cfg.k_cache), v_cache=dev_bf16(cfg.v_cache),
+                               ring_slots=cfg.k_cache.shape[1])
+
+
+def make_prefill(lens, hkv, base, window, sink, seed, klens=None):
+    """A seeded contiguous varlen prefill (workloads.configs.Prefill): bf16 ~N(0,1) Q/K/V,
+    optional ~N(0,1) sinks; queries bottom-right aligned to their keys."""
+    from workloads import configs, synth
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    klens = lens if klens is None else klens
+    cuk = np.concatenate([[0], np.cumsum(klens)]).astype(np.int32)
+    q = configs.bf16_normal(seed, 1, (int(cu[-1]), 64, 192))
+    k = configs.bf16_normal(seed, 2, (int(cuk[-1]), hkv, 192))
+    v = configs.bf16_normal(seed, 3, (int(cuk[-1]), hkv, 128))
+    s = synth.normal_f32(synth.stream_seed(seed, 4), (64,)) if sink else None
+    return configs.Prefill(configs.Layer("swa" if window else "global", hkv, base, window, s), q, k, v, cu, cuk)
+
+
+def check_prefill(cfg, rows=None, what="", **kw):
+    """GPU prefill of cfg against the oracle on `rows` (default all); returns the errors."""
+    import oracle
+    out, lse = prefill_cfg(cfg, **kw)
+    ro, rl = oracle.prefill(cfg, rows=rows)
+    if rows is not None:
+        import torch
+        idx = torch.as_tensor(np.asarray(rows), dtype=torch.long, device=out.device)
+        out, lse = out[idx], lse[idx]
+    return parity(out, lse, ro, rl, what)

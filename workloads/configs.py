@@ -240,17 +240,19 @@ def decode_contexts(seed: int = BASE_SEED + 3, B: int = 64) -> np.ndarray:
     return synth.randint(synth.stream_seed(seed, 0), B, 4096, 65536).astype(np.int32)
 
 
-def decode_batch(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536)) -> tuple[Decode, Decode]:
-    """Decode step, batch B: the SWA layer over a 128-slot ring, the global layer over
-    a paged cache (page 128) with contexts uniform in ctx_range."""
+def decode_batch(seed: int = BASE_SEED + 3, B: int = 64, ctx_range=(4096, 65536),
+                 ring_slots: int = RING) -> tuple[Decode, Decode]:
+    """Decode step, batch B: the SWA layer over a ring of `ring_slots` slots per sequence
+    (128 by default; every slot holds a key), the global layer over a paged cache (page 128)
+    with contexts uniform in ctx_range."""
     if ctx_range == (4096, 65536) and B == 64:
         ctx = decode_contexts(seed, B)
     else:
         ctx = synth.randint(synth.stream_seed(seed, 0), B, *ctx_range).astype(np.int32)
     Ls = swa_layer(synth.normal_f32(synth.stream_seed(seed, 4), (HQ,)))
     swa = Decode(Ls, bf16_normal(seed, 1, (B, HQ, DQK)), ctx,
-                 cached_keys(seed, 2, (B, RING, 8, DQK)), bf16_normal(seed, 3, (B, RING, 8, DV)),
-                 name=f"swa_decode_b{B}_ring128")
+                 cached_keys(seed, 2, (B, ring_slots, 8, DQK)), bf16_normal(seed, 3, (B, ring_slots, 8, DV)),
+                 name=f"swa_decode_b{B}_ring{ring_slots}")
     bt, pool = paged_layout(seed, 10, ctx)
     Lg = global_layer()
     glb = Decode(Lg, bf16_normal(seed, 11, (B, HQ, DQK)), ctx,
@@ -320,9 +322,10 @@ def sample_rows(seed: int, n_total: int, n_sample: int, always=()) -> np.ndarray
 
 
 def chunked_prefill(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int = 8192,
-            n_sample: int = 1024) -> tuple[Chunked, Chunked]:
+            n_sample: int = 1024, ring_slots: int = RING) -> tuple[Chunked, Chunked]:
     """Chunked prefill: `chunk` new tokens after a `prefix`-token cached prefix, for the
-    global layer (paged cache) and the matching SWA layer (ring holding the prefix tail)."""
+    global layer (paged cache) and the matching SWA layer (a ring of `ring_slots` slots
+    holding the prefix tail)."""
     start = np.array([prefix], np.int32)
     cu = np.array([0, chunk], np.int32)
     ctx = np.array([prefix + chunk], np.int32)
@@ -343,15 +346,15 @@ def chunked_prefill(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int 
                   bf16_normal(seed, 3, (chunk, 4, DV)), cu, start, kc, vc, block_table=bt,
                   sample_rows=rows, name=f"global_chunk_{chunk}_on_{prefix}")
     Ls = swa_layer(synth.normal_f32(synth.stream_seed(seed, 24), (HQ,)))
-    ring_k = np.zeros((1, RING, 8, DQK), np.uint16)
-    ring_v = np.zeros((1, RING, 8, DV), np.uint16)
-    tail = min(prefix, RING)
+    ring_k = np.zeros((1, ring_slots, 8, DQK), np.uint16)
+    ring_v = np.zeros((1, ring_slots, 8, DV), np.uint16)
+    tail = min(prefix, ring_slots)
     tk = cached_keys(seed, 25, (tail, 8, DQK))
     tv = bf16_normal(seed, 26, (tail, 8, DV))
     for j in range(tail):
         p = prefix - tail + j
-        ring_k[0, p % RING] = tk[j]
-        ring_v[0, p % RING] = tv[j]
+        ring_k[0, p % ring_slots] = tk[j]
+        ring_v[0, p % ring_slots] = tv[j]
     swa = Chunked(Ls, bf16_normal(seed, 21, (chunk, HQ, DQK)), bf16_normal(seed, 22, (chunk, 8, DQK)),
                   bf16_normal(seed, 23, (chunk, 8, DV)), cu, start, ring_k, ring_v,
                   sample_rows=rows, name=f"swa_chunk_{chunk}_on_{prefix}")
