@@ -18,6 +18,7 @@ fraction of the roofline max(FLOP / bf16 peak, bytes / HBM peak)).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -39,11 +40,10 @@ FLOP_PER_PAIR = 2 * 192 + 2 * 128  # QK^T and PV per visible (query head, key) p
 # The step's dominant kernel (about 96% of the step's device time in the ncu launch list).
 DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
-# workload.  Measured with one ncu capture of the kernel on a 2 x 4096-token sliding-window
-# prefill (inputs larger than L2): 249.66 MB read + 104.12 MB written, scaled by tokens to the
-# 40696-token workload (the kernel's traffic is proportional to tokens).  Set to None whenever
-# the kernel changes after the capture.
-TRAFFIC_BYTES = {"prefill_swa_kernel": int((249.656832e6 + 104.123392e6) * 40696 / 8192)}
+# workload, from one ncu capture of the kernel on a 2 x 4096-token sliding-window prefill
+# (inputs larger than L2) scaled by tokens to the 40696-token workload (the kernel's traffic
+# is proportional to tokens).  None until the current kernel has been captured.
+TRAFFIC_BYTES = {"prefill_swa_kernel": None}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
@@ -101,6 +101,15 @@ def chunked_counts(cfg):
     if cfg.paged:
         by += n * L.num_kv_heads * (192 + 128) * 2 * 2
     return pairs * 64 * FLOP_PER_PAIR, by
+
+
+def verify_counts(cfg):
+    """Draft verification: the chunk's counts (queries and outputs once, every key the drafts
+    attend once per KV head) plus the append of the drafts' keys and values to the cache."""
+    flops, by = chunked_counts(cfg)
+    if not cfg.paged:  # chunked_counts already counts the append of a paged layer
+        by += int(cfg.cu_new[-1]) * cfg.layer.num_kv_heads * (192 + 128) * 2 * 2
+    return flops, by
 
 
 def roofline_us(flops, by, hbm, tf):
@@ -389,6 +398,61 @@ class Chunked:
                                 lse=self.lse, workspace=self.ws)
 
 
+class Verify:
+    """Draft verification through the decode kernel: the q_len draft tokens of every sequence
+    are appended to the cache (the paged cache, or a ring of 144 slots holding the prefix tail
+    and the drafts), then scored by one decode call with q_len query rows per sequence."""
+
+    def __init__(self, cfg, ring_slots=144):
+        import torch
+        import global_attention_attn_b200 as M
+        self.cfg, self.M = cfg, M
+        L = cfg.layer
+        lens = np.diff(cfg.cu_new)
+        self.q_len = int(lens[0])
+        B = len(cfg.start)
+        self.q, self.k, self.v = dev_bf16(cfg.q), dev_bf16(cfg.k_new), dev_bf16(cfg.v_new)
+        self.pos = dev_i32(np.repeat(cfg.start, self.q_len) + np.tile(np.arange(self.q_len), B))
+        self.seq = dev_i32(np.repeat(np.arange(B), self.q_len))
+        ctx = (cfg.start + self.q_len).astype(np.int32)
+        self.ctx, self.max_len = dev_i32(ctx), int(ctx.max())
+        if cfg.paged:
+            self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
+            self.extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
+                              num_pages=cfg.k_cache.shape[0])
+        else:
+            rk, rv = configs.ring_from_chunk(cfg, ring_slots)
+            self.kc, self.vc = dev_bf16(rk), dev_bf16(rv)
+            self.extra = dict(cache_kind=M.MIMO_CACHE_RING, ring_slots=ring_slots)
+        self.sink = dev_f32(L.sink)
+        n = B * self.q_len
+        self.out = torch.empty((n, 64, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((n, 64), dtype=torch.float32, device="cuda")
+        w = M.decode_workspace_size(B, self.max_len, L.num_kv_heads, L.window, self.q_len)
+        self.ws = torch.empty(max(w, 256), dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        M, L = self.M, self.cfg.layer
+        M.mimo_kv_append(self.k, self.v, self.pos, self.seq, rope_base=L.rope_base, k_cache=self.kc, v_cache=self.vc,
+                         num_seqs=len(self.cfg.start), **self.extra)
+        M.mimo_attn_decode(self.q, self.ctx, max_seq_len=self.max_len, num_kv_heads=L.num_kv_heads,
+                           rope_base=L.rope_base, window=L.window, k_cache=self.kc, v_cache=self.vc, sink=self.sink,
+                           out=self.out, lse=self.lse, workspace=self.ws, q_len=self.q_len, **self.extra)
+
+
+def host_call_us(call, n=50):
+    """Host wall time of one call (the Python binding's marshalling, the library's validation,
+    tensor-map encoding and launches), the device kept busy by nothing else."""
+    import torch
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        call()
+    dt = (time.perf_counter() - t0) / n
+    torch.cuda.synchronize()
+    return dt * 1e6
+
+
 def graph_replay_us(call, flush_buf, n=100):
     """Device time of one call when n calls are replayed from a CUDA graph (no host launch
     overhead between them), each after an L2 flush: a graph of n x (flush + call) minus a
@@ -600,68 +664,51 @@ def main():
         per = {}
         flush = l2_flusher()
         flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def measure(name, call, counts, iters, small):
+            """One per-config entry: event-timed calls (L2 flushed before each call for the
+            small workloads, whose inputs fit in L2), and for the microsecond-scale ones also
+            the device time per call in a CUDA-graph replay and the host time the Python call
+            itself takes (marshalling, tensor-map encoding, launches)."""
+            flops, by = counts
+            for _ in range(3):
+                call()
+            ms = event_time_ms(call, iters, flush=flush if small else None) / iters
+            e = _entry(flops, by, ms, hbm, tf_burst, "L2 flushed before each call" if small else "inputs larger than L2")
+            if small:
+                e["graph_replay"] = graph_entry(call, flush_buf, e["roofline_us"])
+                e["host_us_per_call"] = host_call_us(call)
+            per[name] = e
+
         c0 = configs.swa_prefill_s512()
-        f0, b0 = prefill_counts(c0)
-        w0 = Prefill(c0)
-        for _ in range(3):
-            w0()
-        t0 = event_time_ms(w0, 50, flush=flush) / 50
-        per["swa_prefill_s512"] = _entry(f0, b0, t0, hbm, tf_burst, "L2 flushed before each call")
-        per["swa_prefill_s512"]["graph_replay"] = graph_entry(w0, flush_buf, per["swa_prefill_s512"]["roofline_us"])
-        del w0
+        measure("swa_prefill_s512", Prefill(c0), prefill_counts(c0), 50, True)
         c2 = configs.global_causal_prefill()
-        f2, b2 = prefill_counts(c2)
-        w2 = Prefill(c2)
-        for _ in range(3):
-            w2()
-        t2 = event_time_ms(w2, 10) / 10
-        per["global_prefill_s16384"] = _entry(f2, b2, t2, hbm, tf_burst, "inputs larger than L2")
-        del w2, c2
+        measure("global_prefill_s16384", Prefill(c2), prefill_counts(c2), 10, False)
+        del c2
         torch.cuda.empty_cache()
         sw, gl = configs.decode_batch()
-        for name, c, fl in (("swa_decode_b64_ring128", sw, flush), ("global_decode_b64_paged128", gl, None)):
-            fd, bd = decode_counts(c)
-            w = Decode(c)
-            for _ in range(3):
-                w()
-            td = event_time_ms(w, 20, flush=fl) / 20
-            e = _entry(fd, bd, td, hbm, tf_burst, "L2 flushed before each call" if fl else "inputs larger than L2")
-            e["GB/s"] = bd / (td * 1e-3) / 1e9
-            if fl:
-                e["graph_replay"] = graph_entry(w, flush_buf, e["roofline_us"])
-            per[name] = e
-            del w
+        measure("swa_decode_b64_ring128", Decode(sw), decode_counts(sw), 20, True)
+        measure("global_decode_b64_paged128", Decode(gl), decode_counts(gl), 20, False)
+        # the SGLang window of the query plus 128 previous keys, decoded from 144-slot rings
+        sw144, _ = configs.decode_batch(ring_slots=144)
+        sw144.layer = dataclasses.replace(sw144.layer, window=129)
+        measure("swa_decode_b64_ring144_window129", Decode(sw144), decode_counts(sw144), 20, True)
+        del sw144
         # the same global decode over an E4M3 cache (per-KV-head scales)
         c8 = configs.decode_fp8(ctx=gl.ctx)
-        fd, bd = decode_counts(c8)
-        w = Decode(c8)
-        for _ in range(3):
-            w()
-        td = event_time_ms(w, 20) / 20
-        per["global_decode_b64_paged128_fp8"] = _entry(fd, bd, td, hbm, tf_burst, "inputs larger than L2")
-        del w, c8
+        measure("global_decode_b64_paged128_fp8", Decode(c8), decode_counts(c8), 20, False)
+        del c8
         torch.cuda.empty_cache()
-        # speculative verification: 4 draft tokens per sequence on the 64-sequence decode caches
+        # speculative verification: 4 draft tokens per sequence on the 64-sequence decode caches,
+        # appended to the cache and scored by the decode kernel in one call
         vg, vs = configs.verify(B=64, q_len=4, decode=gl)
-        for name, c in (("global_verify_b64_q4", vg), ("swa_verify_b64_q4", vs)):
-            fc, bc = chunked_counts(c)
-            w = Chunked(c)
-            for _ in range(3):
-                w()
-            tc = event_time_ms(w, 10, flush=flush) / 10
-            per[name] = _entry(fc, bc, tc, hbm, tf_burst, "L2 flushed before each call")
-            del w
+        measure("global_verify_b64_q4", Verify(vg), verify_counts(vg), 10, False)
+        measure("swa_verify_b64_q4", Verify(vs), verify_counts(vs), 20, True)
         del sw, gl, vg, vs
         torch.cuda.empty_cache()
         g4, s4 = configs.chunked_prefill()
-        for name, c in (("global_chunk_8192_on_120832", g4), ("swa_chunk_8192_on_120832", s4)):
-            fc, bc = chunked_counts(c)
-            w = Chunked(c)
-            for _ in range(3):
-                w()
-            tc = event_time_ms(w, 5) / 5
-            per[name] = _entry(fc, bc, tc, hbm, tf_burst, "inputs larger than L2")
-            del w
+        measure("global_chunk_8192_on_120832", Chunked(g4), chunked_counts(g4), 5, False)
+        measure("swa_chunk_8192_on_120832", Chunked(s4), chunked_counts(s4), 10, True)
         line["per_config"] = per
         line["cpu_baseline"] = cpu_baseline(cfg)
     print(json.dumps(line), flush=True) if rank == 0 else None

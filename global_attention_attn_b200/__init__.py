@@ -31,6 +31,7 @@ MIMO_DTYPE_BF16 = 0
 MIMO_DTYPE_FP8_E4M3 = 1
 MIMO_RING_SLOTS_DEFAULT = 128
 MIMO_RING_SLOTS_MAX = 512
+MIMO_MAX_DRAFTS = 8
 
 NUM_Q_HEADS = 64
 HEAD_DIM_QK = 192
@@ -40,7 +41,8 @@ SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
 V_SCALE = 0.707
 
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_prefill_workspace_size", "mimo_attn_prefill_stall_test", "mimo_attn_decode",
-           "mimo_attn_decode_workspace_size", "mimo_attn_decode_noalloc", "mimo_kv_append", "mimo_last_error",
+           "mimo_attn_decode_workspace_size", "mimo_attn_verify_workspace_size", "mimo_attn_decode_noalloc",
+           "mimo_kv_append", "mimo_last_error",
            "mimo_status_poll", "mimo_version", "mimo_window_from_left_right")
 DECODE_NOALLOC_MAX_BYTES = 16 << 20
 
@@ -69,7 +71,7 @@ class MimoDecodeArgs(C.Structure):
                 ("block_table", _P), ("max_pages", C.c_int), ("num_pages", C.c_int), ("out", _P), ("lse", _P),
                 ("workspace", _P), ("workspace_bytes", C.c_size_t), ("ev_kernel_begin", _P),
                 ("ev_kernel_end", _P), ("cache_dtype", C.c_int), ("k_dequant", _P), ("v_dequant", _P),
-                ("ring_slots", C.c_int)]
+                ("ring_slots", C.c_int), ("q_len", C.c_int)]
 
 
 class MimoAppendArgs(C.Structure):
@@ -108,6 +110,8 @@ def lib():
         L.mimo_attn_decode.restype = C.c_int
         L.mimo_attn_decode_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
         L.mimo_attn_decode_workspace_size.restype = C.c_size_t
+        L.mimo_attn_verify_workspace_size.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.mimo_attn_verify_workspace_size.restype = C.c_size_t
         L.mimo_attn_decode_noalloc.argtypes = [C.POINTER(MimoDecodeArgs), _P]
         L.mimo_attn_decode_noalloc.restype = C.c_int
         L.mimo_kv_append.argtypes = [C.POINTER(MimoAppendArgs), _P]
@@ -154,8 +158,10 @@ def prefill_workspace_size(num_seqs: int, total_q: int, total_k: int, num_kv_hea
     return int(lib().mimo_attn_prefill_workspace_size(num_seqs, total_q, total_k, num_kv_heads, cache_kind))
 
 
-def decode_workspace_size(batch: int, max_seq_len: int, num_kv_heads: int, window: int) -> int:
-    return int(lib().mimo_attn_decode_workspace_size(batch, max_seq_len, num_kv_heads, window))
+def decode_workspace_size(batch: int, max_seq_len: int, num_kv_heads: int, window: int, q_len: int = 1) -> int:
+    if q_len == 1:
+        return int(lib().mimo_attn_decode_workspace_size(batch, max_seq_len, num_kv_heads, window))
+    return int(lib().mimo_attn_verify_workspace_size(batch, q_len, max_seq_len, num_kv_heads, window))
 
 
 def _events(pair):
@@ -215,17 +221,21 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
                      cache_kind: int, k_cache, v_cache, block_table=None, num_pages: int = 0, sink=None, out=None,
                      lse=None, workspace=None, softmax_scale: float = SOFTMAX_SCALE, v_scale: float = V_SCALE,
                      stream=None, with_lse: bool = True, kernel_events=None, cache_dtype: int = MIMO_DTYPE_BF16,
-                     k_dequant=None, v_dequant=None, ring_slots: int = 0):
+                     k_dequant=None, v_dequant=None, ring_slots: int = 0, q_len: int = 1):
     """Decode step (see include/mimoattn.h).  kernel_events as for mimo_attn_prefill (around the
     split kernel, not the combine).  ring_slots: slots per sequence of a ring cache (0 = 128).
+    q_len: query tokens per sequence (draft tokens to verify; q holds batch * q_len rows).
     Returns (out, lse)."""
     import torch
-    B = q.shape[0]
+    rows = q.shape[0]
+    if rows % q_len:
+        raise ValueError("q holds batch * q_len rows")
+    B = rows // q_len
     if out is None:
-        out = torch.empty((B, NUM_Q_HEADS, HEAD_DIM_V), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((rows, NUM_Q_HEADS, HEAD_DIM_V), dtype=torch.bfloat16, device=q.device)
     if lse is None and with_lse:
-        lse = torch.empty((B, NUM_Q_HEADS), dtype=torch.float32, device=q.device)
-    need = decode_workspace_size(B, max_seq_len, num_kv_heads, window)
+        lse = torch.empty((rows, NUM_Q_HEADS), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, max_seq_len, num_kv_heads, window, q_len)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     a = MimoDecodeArgs()
@@ -241,7 +251,7 @@ def mimo_attn_decode(q, seq_lens, *, max_seq_len: int, num_kv_heads: int, rope_b
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.ev_kernel_begin, a.ev_kernel_end = _events(kernel_events)
     a.cache_dtype, a.k_dequant, a.v_dequant = cache_dtype, _ptr(k_dequant), _ptr(v_dequant)
-    a.ring_slots = int(ring_slots)
+    a.ring_slots, a.q_len = int(ring_slots), int(q_len)
     _check(lib().mimo_attn_decode(C.byref(a), _stream(stream)))
     return out, lse
 

@@ -194,12 +194,30 @@ int make_map(const char* fn, EncodeTiledFn enc, CUtensorMap* m, const void* base
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Keys a decode unit range covers at most: the window of the earliest of q_len query rows
+// reaches q_len - 1 keys further back than the last row's.
+int decode_unit_keys(int max_seq_len, int window, int q_len) {
+  if (window <= 0) return max_seq_len;
+  const long w = long(window) + q_len - 1;
+  return w < max_seq_len ? int(w) : max_seq_len;
+}
+
 // Keys per decode split (a multiple of the kernel's 16-key tile).
-int decode_split_len(int max_seq_len, int window) {
-  const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
-  if (n <= 256) return 256;
-  if (n <= 8192) return 512;
+int decode_split_len(int unit_keys) {
+  if (unit_keys <= 256) return 256;
+  if (unit_keys <= 8192) return 512;
   return 1024;
+}
+
+// Split-KV partials of a decode call: (batch * q_len) query rows x 64 heads x splits.
+size_t decode_workspace(int batch, int q_len, int max_seq_len, int window) {
+  if (batch <= 0 || max_seq_len <= 0 || q_len <= 0) return 0;
+  const int n = decode_unit_keys(max_seq_len, window, q_len);
+  const int split = decode_split_len(n);
+  const int ns = (n + split - 1) / split;
+  if (ns <= 1) return 0;
+  const size_t rows = size_t(batch) * q_len;
+  return round256(rows * kHq * ns * kDv * 4) + round256(rows * kHq * ns * 2 * 4);
 }
 
 }  // namespace
@@ -229,19 +247,21 @@ size_t mimo_attn_prefill_workspace_size(int num_seqs, int total_q, int total_k, 
   const size_t cs = round256(size_t(total_q) * kHalf * 8);  // (cos, sin) per query row and frequency
   if (cache_kind == MIMO_CACHE_RING) {
     const size_t rows = size_t(total_k) + 128 * size_t(num_seqs);
-    return round256(rows * num_kv_heads * kDqk * 2) + round256(rows * num_kv_heads * kDv * 2) + cs;
+    return round256(rows * num_kv_heads * kDqk * 2) + round256(rows * num_kv_heads * kDv * 2) +
+           round256(size_t(total_k) * num_kv_heads * kRope * 2) + cs;
   }
   return round256(size_t(total_k) * num_kv_heads * kRope * 2) + cs;
 }
 
 size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int num_kv_heads, int window) {
   (void)num_kv_heads;
-  if (batch <= 0 || max_seq_len <= 0) return 0;
-  const int split = decode_split_len(max_seq_len, window);
-  const int n = window > 0 ? (max_seq_len < window ? max_seq_len : window) : max_seq_len;
-  const int ns = (n + split - 1) / split;
-  if (ns <= 1) return 0;
-  return round256(size_t(batch) * kHq * ns * kDv * 4) + round256(size_t(batch) * kHq * ns * 2 * 4);
+  return decode_workspace(batch, 1, max_seq_len, window);
+}
+
+size_t mimo_attn_verify_workspace_size(int batch, int q_len, int max_seq_len, int num_kv_heads, int window) {
+  (void)num_kv_heads;
+  if (q_len < 1 || q_len > MIMO_MAX_DRAFTS) return 0;
+  return decode_workspace(batch, q_len, max_seq_len, window);
 }
 
 int mimo_kv_append(const mimo_append_args* a, void* stream) {
@@ -310,9 +330,16 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
     return fail(MIMO_ERR_INVALID_ARG, "%s: cache_kind must be MIMO_CACHE_RING or MIMO_CACHE_PAGED", fn);
   int ring_slots = 0;
   if (int rc = ring_slots_of(fn, a->ring_slots, &ring_slots)) return rc;
-  if (a->cache_kind == MIMO_CACHE_RING && (a->layer.window <= 0 || a->layer.window > ring_slots))
-    return fail(MIMO_ERR_INVALID_ARG, "%s: a ring cache of %d slots holds %d positions: window must be in 1..%d", fn,
-                ring_slots, ring_slots, ring_slots);
+  const int q_len = a->q_len == 0 ? 1 : a->q_len;
+  if (q_len < 1 || q_len > MIMO_MAX_DRAFTS)
+    return fail(MIMO_ERR_INVALID_ARG, "%s: q_len must be 0 or 1 (decode) or at most %d draft tokens (got %d)", fn,
+                MIMO_MAX_DRAFTS, a->q_len);
+  if (a->cache_kind == MIMO_CACHE_RING && (a->layer.window <= 0 || long(a->layer.window) + q_len - 1 > ring_slots))
+    return fail(MIMO_ERR_INVALID_ARG,
+                "%s: a ring cache of %d slots holds %d positions: window + q_len - 1 must be in 1..%d (window %d, "
+                "q_len %d)",
+                fn, ring_slots, ring_slots, ring_slots, a->layer.window, q_len);
+  if (a->max_seq_len < q_len) return fail(MIMO_ERR_INVALID_ARG, "%s: max_seq_len is below q_len", fn);
   REQUIRE_PTR(a->q, "q");
   REQUIRE_PTR(a->seq_lens, "seq_lens");
   REQUIRE_PTR(a->k_cache, "k_cache");
@@ -328,7 +355,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
       return fail(MIMO_ERR_INVALID_ARG, "%s: max_pages * 128 is below max_seq_len", fn);
   }
   if (int rc = check_cache_dtype(fn, a->cache_dtype, a->k_dequant, a->v_dequant)) return rc;
-  const size_t need = mimo_attn_decode_workspace_size(a->batch, a->max_seq_len, a->layer.num_kv_heads, a->layer.window);
+  const size_t need = decode_workspace(a->batch, q_len, a->max_seq_len, a->layer.window);
   if (need > 0) {
     if (!a->workspace || a->workspace_bytes < need)
       return fail(MIMO_ERR_WORKSPACE, "%s: workspace of %zu bytes required (got %zu)", fn, need,
@@ -344,7 +371,10 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   {
     const long rows = a->cache_kind == MIMO_CACHE_RING ? long(a->batch) * ring_slots : long(a->num_pages) * kPage;
     const bool fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
-    int rc = make_map(fn, enc, &p.tm_q, a->q, a->batch, kHq, kDqk, 16, 1);
+    // queries [batch * q_len, 64, 192]: a 16-row block is 16 heads of one row (global layers)
+    // or 8 heads of two rows (sliding-window layers)
+    const int G = kHq / a->layer.num_kv_heads;
+    int rc = make_map(fn, enc, &p.tm_q, a->q, long(a->batch) * q_len, kHq, kDqk, G, 16 / G);
     if (!rc) rc = make_map(fn, enc, &p.tm_k, a->k_cache, rows, a->layer.num_kv_heads, kDqk, 1, 16, fp8);
     if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, a->layer.num_kv_heads, kDv, 1, 16, fp8);
     if (rc) return rc;
@@ -353,9 +383,16 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   p.hkv = a->layer.num_kv_heads;
   p.group = kHq / p.hkv;
   p.window = a->layer.window;
-  p.split_len = decode_split_len(a->max_seq_len, a->layer.window);
-  const int n = p.window > 0 ? (a->max_seq_len < p.window ? a->max_seq_len : p.window) : a->max_seq_len;
+  p.q_len = q_len;
+  {
+    int nc = 0;
+    decode_rows(q_len, p.group, &p.n_blocks, &nc, &p.n_rp);
+  }
+  const int n = decode_unit_keys(a->max_seq_len, p.window, q_len);
+  p.split_len = decode_split_len(n);
   p.max_splits = (n + p.split_len - 1) / p.split_len;
+  if (a->cache_kind == MIMO_CACHE_RING && p.max_splits != 1)  // window + q_len - 1 <= 512 keys: one split
+    return fail(MIMO_ERR_INVALID_ARG, "%s: a ring decode takes one split (internal)", fn);
   p.scale_log2 = a->layer.softmax_scale * 1.4426950408889634f;
   p.v_scale = a->layer.v_scale;
   p.sink = a->layer.sink;
@@ -372,7 +409,7 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
   p.lse = a->lse;
   p.ws_o = need ? static_cast<float*>(a->workspace) : nullptr;
   p.ws_ml = need ? reinterpret_cast<float*>(static_cast<char*>(a->workspace) +
-                                            round256(size_t(a->batch) * kHq * p.max_splits * kDv * 4))
+                                            round256(size_t(a->batch) * q_len * kHq * p.max_splits * kDv * 4))
                  : nullptr;
   p.fp8 = a->cache_dtype == MIMO_DTYPE_FP8_E4M3;
   p.k_dequant = a->k_dequant;
@@ -461,6 +498,7 @@ int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsig
   if (rc) return rc;
   uint16_t* ws_k = static_cast<uint16_t*>(a->workspace);
   uint16_t* ws_v = nullptr;
+  uint16_t* ws_rot = nullptr;
   float2* cs_q = nullptr;
   if (mode != kModePaged) {
     const size_t cs_bytes = round256(size_t(a->total_q) * kHalf * 8);
@@ -482,11 +520,17 @@ int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsig
     if ((rc = make_map(fn, enc, &p.tm_k12, a->k, a->total_k, hkv, kDqk, 1, BN))) return rc;
     if ((rc = make_map(fn, enc, &p.tm_v, a->v, a->total_k, hkv, kDv, 1, BN))) return rc;
   } else if (mode == kModeExt) {
+    // [halo | new] copy of K, of V, then the rotated dims of the new keys
     const long rows = long(a->total_k) + 128L * a->num_seqs;
-    ws_v = reinterpret_cast<uint16_t*>(static_cast<char*>(a->workspace) + round256(size_t(rows) * hkv * kDqk * 2));
+    const size_t k_bytes = round256(size_t(rows) * hkv * kDqk * 2), v_bytes = round256(size_t(rows) * hkv * kDv * 2);
+    ws_v = reinterpret_cast<uint16_t*>(static_cast<char*>(a->workspace) + k_bytes);
+    ws_rot = reinterpret_cast<uint16_t*>(static_cast<char*>(a->workspace) + k_bytes + v_bytes);
     if ((rc = make_map(fn, enc, &p.tm_k0, ws_k, rows, hkv, kDqk, 1, BN))) return rc;
     if ((rc = make_map(fn, enc, &p.tm_k12, ws_k, rows, hkv, kDqk, 1, BN))) return rc;
     if ((rc = make_map(fn, enc, &p.tm_v, ws_v, rows, hkv, kDv, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_k0n, ws_rot, a->total_k, hkv, kRope, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_k12n, a->k, a->total_k, hkv, kDqk, 1, BN))) return rc;
+    if ((rc = make_map(fn, enc, &p.tm_vn, a->v, a->total_k, hkv, kDv, 1, BN))) return rc;
   } else {
     const long rows = long(a->num_pages) * kPage;
     if ((rc = make_map(fn, enc, &p.tm_k0, a->k_cache, rows, hkv, kDqk, 1, BN))) return rc;
@@ -531,6 +575,7 @@ int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsig
     r.ring_slots = ring_slots;
     r.ws_k = ws_k;
     r.ws_v = ws_v;
+    r.ws_rot = ws_rot;
     r.total_q = kind == 0 ? a->total_q : 0;
     r.cu_q = a->cu_seqlens_q;
     r.cs_q = cs_q;
@@ -555,7 +600,9 @@ int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsig
     q.cu_k = a->cu_seqlens_k ? a->cu_seqlens_k + s0 : nullptr;
     q.cache_lens = a->cache_lens ? a->cache_lens + s0 : nullptr;
     q.block_table = a->block_table ? a->block_table + long(s0) * a->max_pages : nullptr;
-    cudaError_t e = launch_prefill(q, kind, grid, st);
+    // overlap the first launch with the key pre-pass, unless the caller times the kernel alone
+    const bool pdl = s0 == 0 && mode != kModePaged && !a->ev_kernel_begin && !a->ev_kernel_end;
+    cudaError_t e = launch_prefill(q, kind, grid, st, pdl);
     if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   }
   if (a->ev_kernel_end) {
@@ -589,8 +636,7 @@ int mimo_attn_decode_noalloc(const mimo_decode_args* a, void* stream) {
   const char* fn = "mimo_attn_decode_noalloc";
   if (!a) return fail(MIMO_ERR_INVALID_ARG, "%s: args is NULL", fn);
   if (a->batch > 0 && a->max_seq_len > 0) {
-    const size_t need =
-        mimo_attn_decode_workspace_size(a->batch, a->max_seq_len, a->layer.num_kv_heads, a->layer.window);
+    const size_t need = decode_workspace(a->batch, a->q_len == 0 ? 1 : a->q_len, a->max_seq_len, a->layer.window);
     if (need > MIMO_DECODE_NOALLOC_MAX_BYTES)
       return fail(MIMO_ERR_WORKSPACE,
                   "%s: batch %d x max_seq_len %d needs %zu bytes of split-KV partials; the library's static "

@@ -87,6 +87,7 @@ struct TileInfo {
   int qpos0;                 // position of tile row 0
   int key_lo;                // first key position that exists
   int krow_base, kpos_base;  // contiguous key sources: row of position kpos_base
+  int new_row0, new_pos0;    // ring-cache chunk: row of the first new key in k / v, its position
 };
 
 // Per-CTA copy of the per-sequence quantities the roles need for every tile.
@@ -174,6 +175,8 @@ __device__ __forceinline__ bool locate(const PrefillParams& p, const SeqTable& S
     T.key_lo = max(0, clen - 128);
     T.krow_base = S.k0[lo] + 128 * (p.seq_base + lo);
     T.kpos_base = clen - 128;
+    T.new_row0 = S.k0[lo];
+    T.new_pos0 = clen;
   } else {
     T.key_lo = 0;
     T.krow_base = 0;
@@ -281,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         tma_prefetch(&p.tm_k12);
         tma_prefetch(&p.tm_v);
       }
+      // the rotated key copies come from the key pre-pass, which may still be running
+      pdl_wait_prerequisites();
       int mt = 0, jj = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok; w += gridDim.x) {
@@ -716,13 +721,29 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
         tma_prefetch(&p.tm_k12);
         tma_prefetch(&p.tm_v);
         tma_prefetch(&p.tm_cs);
+        if (p.mode == kModeExt) {
+          tma_prefetch(&p.tm_k0n);
+          tma_prefetch(&p.tm_k12n);
+          tma_prefetch(&p.tm_vn);
+        }
       }
+      // the rotated key copies and the cos/sin rows come from the key pre-pass, which may
+      // still be running: everything before this point (barriers, tensor memory, the
+      // sequence table) overlapped it
+      pdl_wait_prerequisites();
       bool ok = true;
       int mt = 0;
       for (int w = blockIdx.x; ok; w += gridDim.x, ++mt) {
         TileInfo T;
         if (!locate<0>(p, S, w, T)) break;
-        const int row = T.krow_base + (T.qpos0 - 128 - T.kpos_base);
+        // a ring-cache chunk's tile whose window starts inside the chunk reads the new keys
+        // directly; the others (and every other mode) read the rows T.krow_base refers to
+        const int kt0 = T.qpos0 - 128;
+        const bool direct = p.mode == kModeExt && kt0 >= T.new_pos0;
+        const int row = direct ? T.new_row0 + (kt0 - T.new_pos0) : T.krow_base + (kt0 - T.kpos_base);
+        const CUtensorMap* mk0 = direct ? &p.tm_k0n : &p.tm_k0;
+        const CUtensorMap* mk12 = direct ? &p.tm_k12n : &p.tm_k12;
+        const CUtensorMap* mv = direct ? &p.tm_vn : &p.tm_v;
         if (lane == 0) {
           if (p.withhold_q) break;  // failure-detection test: no query tile ever arrives
           const int b = mt & 1;
@@ -737,15 +758,15 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
           if (mt >= 1 && !(ok = mbar_wait(k_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
           const uint32_t kdst = sbase + Ly::kOffK;
           mbar_expect_tx(k_full, 3 * Ly::kKChunk);
-          tma_load_3d(kdst, &p.tm_k0, k_full, 0, T.g, row);
-          tma_load_3d(kdst + Ly::kKChunk, &p.tm_k12, k_full, 64, T.g, row);
-          tma_load_3d(kdst + 2 * Ly::kKChunk, &p.tm_k12, k_full, 128, T.g, row);
+          tma_load_3d(kdst, mk0, k_full, 0, T.g, row);
+          tma_load_3d(kdst + Ly::kKChunk, mk12, k_full, 64, T.g, row);
+          tma_load_3d(kdst + 2 * Ly::kKChunk, mk12, k_full, 128, T.g, row);
         } else {
           if (mt >= 1 && !(ok = mbar_wait(v_empty, (mt - 1) & 1, abort_flag, status, MIMO_STATUS_TIMEOUT, p.wait_ns))) break;
           const uint32_t vdst = sbase + Ly::kOffV;
           mbar_expect_tx(v_full, 2 * Ly::kVChunk);
-          tma_load_3d(vdst, &p.tm_v, v_full, 0, T.g, row);
-          tma_load_3d(vdst + Ly::kVChunk, &p.tm_v, v_full, 64, T.g, row);
+          tma_load_3d(vdst, mv, v_full, 0, T.g, row);
+          tma_load_3d(vdst + Ly::kVChunk, mv, v_full, 64, T.g, row);
         }
       }
       if (!ok) {
@@ -1148,29 +1169,32 @@ __device__ __forceinline__ int query_position(const RopeKParams& p, long row) {
   return ctx - qlen + int(row - p.cu_q[lo]);
 }
 
-// contig: one thread per (row, u = frequencies 8u..8u+7).  For key rows it writes the
-// rotated dims 0..63 (fp16) of all HKV heads into ws_k: the heads share the row's
-// position, so the 8 (cos, sin) pairs are computed once, and the loads of every head are
-// issued before the trig so that their latency overlaps it.  For query rows (when cs_q is
-// set) it writes the same 8 pairs at the query's position, reusing the key's pairs when
-// the two positions agree (prefill without a cache).
+// contig: one warp per key row.  Lane j computes frequency j's (cos, sin) at the row's
+// position once; lane l rotates chunk pair (head l / 4, u = l % 4) of dims 0..63 with the
+// pairs of frequencies 8u..8u+7 taken from the lanes that hold them, and writes it (fp16)
+// into ws_k.  The loads are issued before the trig so that their latency overlaps it.  For
+// query rows (when cs_q is set) the same warp writes the row's (cos, sin) at the query's
+// position, reusing the key's when the two positions agree (prefill without a cache).  One
+// sine / cosine per lane keeps the latency of a short call low (eight per thread before).
 template <int HKV>
-__global__ void __launch_bounds__(256, 2) rope_k_contig_kernel(const RopeKParams p) {
-  const long gt = long(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long row = gt >> 2;
-  const int u = int(gt & 3);
+__global__ void __launch_bounds__(256) rope_k_contig_kernel(const RopeKParams p) {
+  static_assert(HKV * 4 <= 32, "one rotated chunk pair per lane");
+  pdl_launch_dependents();
+  const long row = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   const bool key_row = row < p.total_k;
   const bool q_row = p.cs_q && row < p.total_q;
-  if (!key_row && !q_row) return;
-  uint4 a[HKV], b[HKV];
+  if (!key_row && !q_row) return;  // warp-uniform: one row per warp
   int pos_k = 0;
-  float2 cs[8];
+  float c_j = 0.f, s_j = 0.f;
   if (key_row) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.k + row * HKV * kDqk) + u;
-#pragma unroll
-    for (int g = 0; g < HKV; ++g) {
-      a[g] = __ldg(src + g * (kDqk / 8));
-      b[g] = __ldg(src + g * (kDqk / 8) + 4);
+    const int g = lane >> 2, u = lane & 3;
+    const bool act = g < HKV;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    const uint4* src = reinterpret_cast<const uint4*>(p.k + (row * HKV + g) * kDqk) + u;
+    if (act) {
+      a = __ldg(src);
+      b = __ldg(src + 4);
     }
     int lo = 0, hi = p.num_seqs;  // find s with cu_k[s] <= row < cu_k[s+1]
     while (hi - lo > 1) {
@@ -1178,27 +1202,26 @@ __global__ void __launch_bounds__(256, 2) rope_k_contig_kernel(const RopeKParams
       if (p.cu_k[mid] <= row) lo = mid; else hi = mid;
     }
     pos_k = (p.cache_lens ? p.cache_lens[lo] : 0) + int(row - p.cu_k[lo]);
+    rope_cos_sin(pos_k, p.rope.inv_freq[lane], &c_j, &s_j);
+    float2 cs[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) rope_cos_sin(pos_k, p.rope.inv_freq[8 * u + i], &cs[i].x, &cs[i].y);
-    uint4* dst = reinterpret_cast<uint4*>(p.ws_k + row * HKV * kRope) + u;
-    float amax = 0.f;
-#pragma unroll
-    for (int g = 0; g < HKV; ++g) {
-      rope_chunk_pair_cs(a[g], b[g], cs, amax);
-      dst[g * (kRope / 8)] = a[g];
-      dst[g * (kRope / 8) + 4] = b[g];
+    for (int f = 0; f < 8; ++f) {
+      cs[f].x = __shfl_sync(0xffffffffu, c_j, 8 * u + f);
+      cs[f].y = __shfl_sync(0xffffffffu, s_j, 8 * u + f);
     }
-    if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
+    if (act) {
+      float amax = 0.f;
+      rope_chunk_pair_cs(a, b, cs, amax);
+      if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
+      uint4* dst = reinterpret_cast<uint4*>(p.ws_k + (row * HKV + g) * kRope) + u;
+      dst[0] = a;
+      dst[4] = b;
+    }
   }
   if (q_row) {
     const int pos_q = query_position(p, row);
-    if (!key_row || pos_q != pos_k) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) rope_cos_sin(pos_q, p.rope.inv_freq[8 * u + i], &cs[i].x, &cs[i].y);
-    }
-    float4* d = reinterpret_cast<float4*>(p.cs_q + row * kHalf + 8 * u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = make_float4(cs[2 * i].x, cs[2 * i].y, cs[2 * i + 1].x, cs[2 * i + 1].y);
+    if (!key_row || pos_q != pos_k) rope_cos_sin(pos_q, p.rope.inv_freq[lane], &c_j, &s_j);
+    p.cs_q[row * kHalf + lane] = make_float2(c_j, s_j);
   }
 }
 
@@ -1214,6 +1237,7 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
   static_assert(HKV * 4 <= 32, "one rotated chunk pair per lane");
   constexpr int kKRow = HKV * kDqk / 8;  // uint4 of one position's keys (all heads)
   constexpr int kVRow = HKV * kDv / 8;
+  pdl_launch_dependents();
   const long wid = (long(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long rows = long(p.total_k) + 128L * p.num_seqs;
@@ -1260,6 +1284,10 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
     } else {
       const long row = p.cu_k[s] + (i - 128);
       pos_k = clen + (i - 128);
+      // every new row: its rotated dims 0..63 into ws_rot (the tiles whose window starts inside
+      // the chunk read those with k and v); the first kExtFullRows rows also whole into the
+      // ext copy, for the tiles whose window reaches back into the halo
+      const bool full_row = i - 128 < kExtFullRows;  // warp-uniform
       const uint4* ks = reinterpret_cast<const uint4*>(p.k + row * HKV * kDqk);
       const uint4* vs = reinterpret_cast<const uint4*>(p.v + row * HKV * kDv);
       // rotated pair of this lane, the plain key chunks (dims 64..191) and the value
@@ -1271,13 +1299,15 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
         ra = __ldg(ks + pg * (kDqk / 8) + pu);
         rb = __ldg(ks + pg * (kDqk / 8) + pu + 4);
       }
+      if (full_row) {
 #pragma unroll
-      for (int t = 0; t < kPlain; ++t) {
-        const int c = lane + 32 * t;
-        kp[t] = __ldg(ks + (c >> 4) * (kDqk / 8) + 8 + (c & 15));
+        for (int t = 0; t < kPlain; ++t) {
+          const int c = lane + 32 * t;
+          kp[t] = __ldg(ks + (c >> 4) * (kDqk / 8) + 8 + (c & 15));
+        }
+#pragma unroll
+        for (int t = 0; t < kVal; ++t) vv[t] = __ldg(vs + lane + 32 * t);
       }
-#pragma unroll
-      for (int t = 0; t < kVal; ++t) vv[t] = __ldg(vs + lane + 32 * t);
       rope_cos_sin(pos_k, p.rope.inv_freq[lane], &c_j, &s_j);
       have_cs = true;
       float2 cs[8];
@@ -1290,16 +1320,23 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
         float amax = 0.f;
         rope_chunk_pair_cs(ra, rb, cs, amax);
         if (amax > kF16Max) atomicOr(p.status, MIMO_STATUS_RANGE);
-        kd[pg * (kDqk / 8) + pu] = ra;
-        kd[pg * (kDqk / 8) + pu + 4] = rb;
+        uint4* rot = reinterpret_cast<uint4*>(p.ws_rot + (row * HKV + pg) * kRope) + pu;
+        rot[0] = ra;
+        rot[4] = rb;
+        if (full_row) {
+          kd[pg * (kDqk / 8) + pu] = ra;
+          kd[pg * (kDqk / 8) + pu + 4] = rb;
+        }
       }
+      if (full_row) {
 #pragma unroll
-      for (int t = 0; t < kPlain; ++t) {
-        const int c = lane + 32 * t;
-        kd[(c >> 4) * (kDqk / 8) + 8 + (c & 15)] = kp[t];
+        for (int t = 0; t < kPlain; ++t) {
+          const int c = lane + 32 * t;
+          kd[(c >> 4) * (kDqk / 8) + 8 + (c & 15)] = kp[t];
+        }
+#pragma unroll
+        for (int t = 0; t < kVal; ++t) vd[lane + 32 * t] = vv[t];
       }
-#pragma unroll
-      for (int t = 0; t < kVal; ++t) vd[lane + 32 * t] = vv[t];
     }
   }
   if (q_row) {
@@ -1314,7 +1351,7 @@ cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s) {
   const long qrows = p.cs_q ? long(p.total_q) : 0;
   if (p.mode == kModeContig) {
     const long rows = long(p.total_k) > qrows ? long(p.total_k) : qrows;
-    const long blocks = (rows * 4 + 255) / 256;
+    const long blocks = (rows * 32 + 255) / 256;
     if (blocks == 0) return cudaSuccess;
     if (p.hkv == 8) rope_k_contig_kernel<8><<<unsigned(blocks), 256, 0, s>>>(p);
     else rope_k_contig_kernel<4><<<unsigned(blocks), 256, 0, s>>>(p);
@@ -1332,20 +1369,30 @@ cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s) {
 int prefill_rows_per_tile(int kind) { return kind == 0 ? Cfg<0>::R : Cfg<1>::R; }
 int prefill_key_tile(int kind) { return kind == 0 ? Cfg<0>::BN : Cfg<1>::BN; }
 
-cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s) {
+cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s, bool pdl) {
   if (grid <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
   if (kind == 0) {
     cudaError_t e = cudaFuncSetAttribute(prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SwaLayout::kAlloc);
     if (e != cudaSuccess) return e;
-    prefill_swa_kernel<<<grid, kSwaThreads, SwaLayout::kAlloc, s>>>(p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Layout<1>::kAlloc);
-    if (e != cudaSuccess) return e;
-    prefill_kernel<1><<<grid, kThreads, Layout<1>::kAlloc, s>>>(p);
+    cfg.blockDim = dim3(kSwaThreads);
+    cfg.dynamicSmemBytes = SwaLayout::kAlloc;
+    return cudaLaunchKernelEx(&cfg, prefill_swa_kernel, p);
   }
-  return cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Layout<1>::kAlloc);
+  if (e != cudaSuccess) return e;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Layout<1>::kAlloc;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<1>, p);
 }
 
 }  // namespace mimo

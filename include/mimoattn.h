@@ -203,17 +203,23 @@ MIMO_API int mimo_attn_prefill_stall_test(const mimo_prefill_args* args, void* s
                                           unsigned long long wait_limit_ns);
 
 /*
- * Decode: one query token per sequence.  Token s sits at position
- * seq_lens[s] - 1 and the cache already holds positions 0 .. seq_lens[s]-1
- * (append the token with mimo_kv_append first).  Sliding-window layers use a
- * ring cache (the last ring_slots positions are kept; window in 1..ring_slots),
+ * Decode: q_len query tokens per sequence, the last q_len positions of its context
+ * (q_len = 1: one decode step; 2..MIMO_MAX_DRAFTS: draft tokens of speculative decoding
+ * scored in one pass, as the serving pages run it: vLLM recipe page, DFlash; SGLang
+ * cookbook page; radixark miles docs section 4.2, EAGLE with 4 draft tokens).  Query
+ * row s * q_len + i sits at position seq_lens[s] - q_len + i and sees the keys up to its
+ * own position (and, with a window, the window before it): draft i sees the context and
+ * drafts 0..i.  The cache already holds positions 0 .. seq_lens[s]-1, the drafts
+ * included (append them with mimo_kv_append first).  Sliding-window layers use a ring
+ * cache (the last ring_slots positions are kept: window + q_len - 1 <= ring_slots),
  * global layers a paged cache (gaudi-cookbook "MiMo-V2.6-Flash-RL", "Launch":
  * window-sized KV for the sliding layers, blocks of 128 positions).
  *
- * Layouts: q [batch, 64, 192] bf16 pre-RoPE; out [batch, 64, 128] bf16;
- * lse [batch, 64] fp32 or NULL.  max_seq_len is a host-side upper bound of
- * seq_lens (it sizes the split-KV grid and the workspace).
+ * Layouts: q [batch * q_len, 64, 192] bf16 pre-RoPE; out [batch * q_len, 64, 128] bf16;
+ * lse [batch * q_len, 64] fp32 or NULL.  max_seq_len is a host-side upper bound of
+ * seq_lens (it sizes the split-KV grid and the workspace); every seq_lens[s] >= q_len.
  */
+#define MIMO_MAX_DRAFTS 8
 typedef struct {
   mimo_layer layer;
   int batch;
@@ -240,10 +246,16 @@ typedef struct {
   const float* k_dequant;   /* FP8: device fp32 [num_kv_heads] key scales, else NULL */
   const float* v_dequant;   /* FP8: device fp32 [num_kv_heads] value scales, else NULL */
   int ring_slots;           /* MIMO_CACHE_RING: slots per sequence of the ring (0 = 128) */
+  int q_len;                /* query tokens per sequence: 0 or 1 (decode), up to MIMO_MAX_DRAFTS */
 } mimo_decode_args;
 
-/* Bytes of workspace mimo_attn_decode needs (split-KV partials). */
+/* Bytes of workspace mimo_attn_decode needs (split-KV partials) for one query token per
+ * sequence. */
 MIMO_API size_t mimo_attn_decode_workspace_size(int batch, int max_seq_len, int num_kv_heads, int window);
+
+/* The same for q_len query tokens per sequence (0 for q_len outside 1..MIMO_MAX_DRAFTS). */
+MIMO_API size_t mimo_attn_verify_workspace_size(int batch, int q_len, int max_seq_len, int num_kv_heads,
+                                                int window);
 
 MIMO_API int mimo_attn_decode(const mimo_decode_args* args, void* stream);
 

@@ -37,20 +37,24 @@ def prefill(cfg, rows=None, nthreads=None, online=False):
 
 
 def decode(cfg, seqs=None, nthreads=None):
-    """Oracle for a decode step (workloads.configs.Decode): one query per sequence at ctx-1."""
+    """Oracle for a decode step (workloads.configs.Decode): q_len queries per sequence at
+    positions ctx-q_len .. ctx-1, every key from the cache.  Returns the rows of the selected
+    sequences in order (q_len rows each)."""
     from . import attention
     B = len(cfg.ctx)
+    ql = int(getattr(cfg, "q_len", 1))
     if seqs is None:
         seqs = np.arange(B)
     seqs = np.asarray(seqs, np.int32)
     kw = dict(cache_kind=1, page_size=cfg.k_cache.shape[1], block_table=cfg.block_table) if cfg.paged else \
         dict(cache_kind=2, page_size=cfg.k_cache.shape[1])
     kw.update(cache_dtype=cfg.cache_dtype, k_dequant=cfg.k_dequant, v_dequant=cfg.v_dequant)
-    return attention(q=cfg.q, **_layer_kw(cfg.layer), q_row0=np.arange(B, dtype=np.int32),
-                     q_len=np.ones(B, np.int32), q_pos0=(cfg.ctx - 1).astype(np.int32), sel_seq=seqs,
-                     sel_row=np.zeros(len(seqs), np.int32), new_row0=np.zeros(B, np.int32),
-                     new_pos0=cfg.ctx.astype(np.int32), new_len=np.zeros(B, np.int32),
-                     k_cache=cfg.k_cache, v_cache=cfg.v_cache, nthreads=nthreads, **kw)
+    return attention(q=cfg.q, **_layer_kw(cfg.layer), q_row0=(np.arange(B) * ql).astype(np.int32),
+                     q_len=np.full(B, ql, np.int32), q_pos0=(cfg.ctx - ql).astype(np.int32),
+                     sel_seq=np.repeat(seqs, ql), sel_row=np.tile(np.arange(ql, dtype=np.int32), len(seqs)),
+                     new_row0=np.zeros(B, np.int32), new_pos0=cfg.ctx.astype(np.int32),
+                     new_len=np.zeros(B, np.int32), k_cache=cfg.k_cache, v_cache=cfg.v_cache, nthreads=nthreads,
+                     **kw)
 
 
 def chunked(cfg, rows=None, nthreads=None):

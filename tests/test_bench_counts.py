@@ -83,3 +83,23 @@ def test_chunked_counts_match_enumeration():
         if cfg.paged:
             want += n * L.num_kv_heads * (192 + 128) * 2 * 2  # the append: read and write
         assert by == want
+
+
+def test_verify_counts_match_enumeration():
+    """Draft verification through the decode kernel: every draft row's visible keys, the keys
+    the drafts attend read once per KV head, queries and outputs once, and the drafts' append
+    (read and written) for both layer kinds."""
+    glb, swa = configs.verify(seed=9, B=5, q_len=4, ctx_range=(5, 700))
+    for cfg in (glb, swa):
+        L = cfg.layer
+        pairs = keys = 0
+        for s, st in enumerate(cfg.start):
+            st = int(st)
+            pairs += brute_pairs(range(st, st + 4), range(st + 4), L.window)
+            keys += st + 4 if not L.window else min(st + 4, 4 + L.window - 1)
+        flops, by = bench.verify_counts(cfg)
+        assert flops == pairs * 64 * FLOP_PER_PAIR
+        n = 5 * 4
+        want = n * 64 * (192 * 2 + 128 * 2 + 4) + keys * L.num_kv_heads * (192 + 128) * 2 \
+            + n * L.num_kv_heads * (192 + 128) * 2 * 2
+        assert by == want

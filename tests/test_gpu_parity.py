@@ -13,7 +13,7 @@ import oracle
 from workloads import configs, synth
 
 from .util import (check_prefill, chunked_cfg, decode_cfg, dev_bf16, dev_f32, dev_i32, host_f64, make_prefill, parity,
-                   prefill_cfg)
+                   prefill_cfg, verify_decode_cfg)
 
 pytestmark = pytest.mark.gpu
 
@@ -364,6 +364,33 @@ def test_chunked_swa_window_left_right_128_0():
     parity(out, lse, ro, rl, swa.name)
 
 
+@pytest.mark.parametrize("window", [128, 129])
+def test_chunked_swa_ring_mixed_lengths(window):
+    """Sliding-window chunks over ring caches, many sequences: chunk lengths on both sides of
+    the 128-position halo and of the 144 new rows copied next to it, prefixes shorter and
+    longer than the ring.  Tiles whose window starts inside the chunk read the new keys
+    directly, the others the copy of the halo and the first new keys."""
+    lens = np.array([1, 16, 127, 128, 129, 143, 144, 145, 300, 517], np.int32)
+    starts = np.array([0, 5, 127, 128, 129, 1000, 3, 200, 4096, 77], np.int32)
+    B = len(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    n = int(cu[-1])
+    seed = 60 + window
+    ring_k = np.zeros((B, 128, 8, 192), np.uint16)
+    ring_v = np.zeros((B, 128, 8, 128), np.uint16)
+    tk = configs.cached_keys(seed, 5, (B, 128, 8, 192))
+    tv = configs.bf16_normal(seed, 6, (B, 128, 8, 128))
+    for s in range(B):
+        for p in range(max(0, int(starts[s]) - 128), int(starts[s])):
+            ring_k[s, p % 128], ring_v[s, p % 128] = tk[s, p % 128], tv[s, p % 128]
+    L = configs.Layer("swa", 8, 1e4, window, synth.normal_f32(synth.stream_seed(seed, 4), (64,)))
+    cfg = configs.Chunked(L, configs.bf16_normal(seed, 1, (n, 64, 192)), configs.bf16_normal(seed, 2, (n, 8, 192)),
+                          configs.bf16_normal(seed, 3, (n, 8, 128)), cu, starts, ring_k, ring_v,
+                          name=f"swa ring chunks of mixed lengths, window {window}")
+    out, lse = chunked_cfg(cfg)
+    parity(out, lse, *oracle.chunked(cfg, rows=np.arange(n)), cfg.name)
+
+
 def test_chunked_swa_from_a_256_slot_ring_window_129():
     """The sliding-window chunk reads its 128 halo positions from a ring longer than 128."""
     import dataclasses
@@ -454,6 +481,81 @@ def test_verify_b64_full_scale(dec64):
         out, lse = chunked_cfg(cfg)
         ro, rl = oracle.chunked(cfg, rows=np.arange(64 * 4))
         parity(out, lse, ro, rl, cfg.name)
+
+
+# ----------------------------------------------------------------------------- draft tokens in the decode kernel
+
+@pytest.mark.parametrize("q_len", [2, 3, 4, 5, 8])
+def test_decode_drafts_paged(q_len):
+    """q_len query tokens per sequence over the paged cache: each draft row with its own
+    position, rotary angle and causal limit."""
+    _, gl = configs.decode_batch(seed=710 + q_len, B=10, ctx_range=(q_len, 3000))
+    gl.ctx[:2] = [q_len, q_len + 1]
+    cfg = configs.with_drafts(gl, q_len, seed=711)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), cfg.name)
+
+
+@pytest.mark.parametrize("q_len,ring_slots,window", [(2, 144, 128), (4, 144, 128), (8, 144, 128), (5, 144, 129),
+                                                     (8, 256, 129), (3, 128, 100)])
+def test_decode_drafts_ring(q_len, ring_slots, window):
+    """Draft rows over a ring: the ring keeps window + q_len - 1 positions, so the earliest
+    draft's window is whole after the drafts are appended."""
+    import dataclasses
+    sw, _ = configs.decode_batch(seed=720 + q_len + ring_slots, B=10, ctx_range=(q_len, 3000), ring_slots=ring_slots)
+    sw.layer = dataclasses.replace(sw.layer, window=window)
+    sw.ctx[:3] = [q_len, window, window + q_len]
+    cfg = configs.with_drafts(sw, q_len, seed=721)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), cfg.name)
+
+
+def test_decode_drafts_split_edges_and_window():
+    """Draft rows straddling the 512-key split boundaries (the rows' partials of one split may
+    be empty), and a paged window with a sink."""
+    import dataclasses
+    ctx = np.array([4, 5, 511, 512, 513, 515, 516, 1025, 8195, 8196], np.int32)
+    _, gl = configs.decode_batch(seed=730, B=len(ctx), ctx_range=(4, 5))
+    bt, pool = configs.paged_layout(731, 1, ctx)
+    gl = configs.Decode(gl.layer, gl.q, ctx, configs.cached_keys(731, 2, (pool, 128, 4, 192)),
+                        configs.bf16_normal(731, 3, (pool, 128, 4, 128)), block_table=bt, name="drafts_split_edges")
+    cfg = configs.with_drafts(gl, 4, seed=732)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), "drafts at split boundaries")
+    sink = synth.normal_f32(synth.stream_seed(733, 9), (64,))
+    cfg.layer = dataclasses.replace(cfg.layer, window=1000, sink=sink)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), "drafts, paged window 1000 with sink")
+
+
+@pytest.mark.parametrize("ring", [False, True])
+def test_decode_drafts_fp8(ring):
+    import dataclasses
+    cfg = configs.decode_fp8(seed=740 + ring, B=8, ctx_range=(4, 3000), ring=ring)
+    if ring:  # 128 slots: window + q_len - 1 <= 128
+        cfg.layer = dataclasses.replace(cfg.layer, window=125)
+    cfg = configs.with_drafts(cfg, 4, seed=742)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), cfg.name)
+
+
+@pytest.mark.parametrize("q_len", [2, 4, 8])
+def test_verify_through_the_decode_kernel(q_len):
+    """The verification workloads scored by the decode kernel (drafts appended to the paged
+    cache or to a 144-slot ring, one decode call with q_len rows per sequence) equal the
+    oracle's chunked prefill of the drafts."""
+    glb, swa = configs.verify(seed=750 + q_len, B=12, q_len=q_len, ctx_range=(q_len + 1, 3000))
+    for cfg in (glb, swa):
+        out, lse = verify_decode_cfg(cfg)
+        parity(out, lse, *oracle.chunked(cfg, rows=np.arange(int(cfg.cu_new[-1]))), cfg.name + " (decode kernel)")
+
+
+def test_verify_b64_through_the_decode_kernel(dec64):
+    _, gl = dec64
+    glb, swa = configs.verify(B=64, q_len=4, decode=gl)
+    for cfg in (glb, swa):
+        out, lse = verify_decode_cfg(cfg)
+        parity(out, lse, *oracle.chunked(cfg, rows=np.arange(64 * 4)), cfg.name + " (decode kernel)")
 
 
 def test_decode_matches_last_prefill_row():

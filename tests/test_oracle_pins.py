@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from workloads import synth
+from workloads import configs, synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -469,3 +469,28 @@ def test_oracle_snapshot():
                                    err_msg=name)
         np.testing.assert_allclose(np.asarray(now[name]["lse"]), np.asarray(vals["lse"]), rtol=0, atol=1e-12,
                                    err_msg=name)
+
+
+@pytest.mark.parametrize("paged", [True, False])
+def test_decode_adapter_with_drafts_equals_single_token_decodes(paged):
+    """The decode adapter with q_len query tokens per sequence: draft i of sequence s (position
+    ctx - q_len + i) must equal a one-token decode of the same query over the same cache with
+    the context ending at its position (keys after it are invisible to it; for the ring the
+    slots that then read as older positions lie outside its window)."""
+    import dataclasses
+    sw, gl = configs.decode_batch(seed=61, B=3, ctx_range=(130, 600), ring_slots=144)
+    base = gl if paged else sw
+    q_len = 4
+    cfg = configs.with_drafts(base, q_len, seed=62)
+    o, l = oracle.decode(cfg)
+    assert o.shape[0] == 3 * q_len
+    for s in range(3):
+        for i in range(q_len):
+            one = dataclasses.replace(cfg, q=cfg.q[s * q_len + i:s * q_len + i + 1], q_len=1,
+                                      ctx=np.array([cfg.ctx[s] - q_len + i + 1], np.int32),
+                                      block_table=None if cfg.block_table is None else cfg.block_table[s:s + 1],
+                                      k_cache=cfg.k_cache if paged else cfg.k_cache[s:s + 1],
+                                      v_cache=cfg.v_cache if paged else cfg.v_cache[s:s + 1])
+            o1, l1 = oracle.decode(one)
+            np.testing.assert_array_equal(o[s * q_len + i], o1[0])
+            np.testing.assert_array_equal(l[s * q_len + i], l1[0])

@@ -77,7 +77,7 @@ def decode_cfg(cfg, **kw):
         kc, vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
     return M.mimo_attn_decode(dev_bf16(cfg.q), dev_i32(cfg.ctx), max_seq_len=int(cfg.ctx.max()),
                               num_kv_heads=L.num_kv_heads, rope_base=L.rope_base, window=L.window,
-                              k_cache=kc, v_cache=vc, sink=dev_f32(L.sink), **extra, **kw)
+                              k_cache=kc, v_cache=vc, sink=dev_f32(L.sink), q_len=cfg.q_len, **extra, **kw)
 
 
 def chunked_cfg(cfg):
@@ -135,3 +135,34 @@ def check_prefill(cfg, rows=None, what="", **kw):
         idx = torch.as_tensor(np.asarray(rows), dtype=torch.long, device=out.device)
         out, lse = out[idx], lse[idx]
     return parity(out, lse, ro, rl, what)
+
+
+def verify_decode_cfg(cfg, ring_slots=144):
+    """Draft verification through the decode kernel for a workloads.configs.Chunked whose new
+    rows are q_len draft tokens per sequence: the drafts are appended to the cache (the paged
+    cache, or a ring of ring_slots slots built from the chunk's prefix tail), then scored by
+    one mimo_attn_decode with q_len query tokens per sequence.  Returns (out, lse) for the
+    draft rows in order."""
+    import global_attention_attn_b200 as M
+    from workloads import configs
+    L = cfg.layer
+    lens = np.diff(cfg.cu_new)
+    q_len = int(lens[0])
+    assert np.all(lens == q_len)
+    B = len(cfg.start)
+    seq = np.repeat(np.arange(B), q_len).astype(np.int32)
+    pos = (np.repeat(cfg.start, q_len) + np.tile(np.arange(q_len), B)).astype(np.int32)
+    ctx = (cfg.start + q_len).astype(np.int32)
+    if cfg.paged:
+        kc, vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
+        extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
+                     num_pages=cfg.k_cache.shape[0])
+    else:
+        rk, rv = configs.ring_from_chunk(cfg, ring_slots)
+        kc, vc = dev_bf16(rk), dev_bf16(rv)
+        extra = dict(cache_kind=M.MIMO_CACHE_RING, ring_slots=ring_slots)
+    M.mimo_kv_append(dev_bf16(cfg.k_new), dev_bf16(cfg.v_new), dev_i32(pos), dev_i32(seq), rope_base=L.rope_base,
+                     k_cache=kc, v_cache=vc, num_seqs=B, **extra)
+    return M.mimo_attn_decode(dev_bf16(cfg.q), dev_i32(ctx), max_seq_len=int(ctx.max()), num_kv_heads=L.num_kv_heads,
+                              rope_base=L.rope_base, window=L.window, k_cache=kc, v_cache=vc, sink=dev_f32(L.sink),
+                              q_len=q_len, **extra)

@@ -150,10 +150,11 @@ class Prefill:
 
 @dataclass
 class Decode:
-    """One query token per sequence at position pos[s] = ctx[s]-1 over a cache that
-    already holds positions 0..ctx-1 (SWA: the last RING of them in a ring)."""
+    """q_len query tokens per sequence (one decode step, or draft tokens to verify): query
+    row s * q_len + i at position ctx[s] - q_len + i, over a cache that already holds
+    positions 0..ctx-1 (SWA: the last ring_slots of them in a ring)."""
     layer: Layer
-    q: np.ndarray            # [B, HQ, DQK] (pre-RoPE)
+    q: np.ndarray            # [B * q_len, HQ, DQK] (pre-RoPE)
     ctx: np.ndarray          # int32 [B]
     # ring cache (SWA): [B, RING, Hkv, D]; paged cache (global): [pages, PAGE, Hkv, D]
     k_cache: np.ndarray
@@ -163,6 +164,7 @@ class Decode:
     cache_dtype: int = 0                     # 0: bf16 rows (fp16 rotated dims); 1: E4M3 bytes
     k_dequant: np.ndarray | None = None      # fp32 [Hkv] dequantisation scales (E4M3 caches)
     v_dequant: np.ndarray | None = None
+    q_len: int = 1
 
     @property
     def paged(self) -> bool:
@@ -359,3 +361,27 @@ def chunked_prefill(seed: int = BASE_SEED + 4, prefix: int = 120832, chunk: int 
                   bf16_normal(seed, 23, (chunk, 8, DV)), cu, start, ring_k, ring_v,
                   sample_rows=rows, name=f"swa_chunk_{chunk}_on_{prefix}")
     return glb, swa
+
+
+def with_drafts(cfg: Decode, q_len: int, seed: int) -> Decode:
+    """The same caches scored by q_len query tokens per sequence: fresh ~N(0,1) queries for
+    the last q_len positions of every context (whose keys the cache already holds)."""
+    import dataclasses
+    B = len(cfg.ctx)
+    assert int(cfg.ctx.min()) >= q_len
+    return dataclasses.replace(cfg, q=bf16_normal(seed, 77, (B * q_len, HQ, DQK)), q_len=q_len,
+                               name=f"{cfg.name}_q{q_len}")
+
+
+def ring_from_chunk(cfg: Chunked, ring_slots: int) -> tuple[np.ndarray, np.ndarray]:
+    """A ring of `ring_slots` slots holding the prefix tail of a sliding-window chunk (the
+    positions its 128-slot ring holds, each moved to slot p % ring_slots); other slots zero."""
+    B, R0 = cfg.k_cache.shape[0], cfg.k_cache.shape[1]
+    rk = np.zeros((B, ring_slots) + cfg.k_cache.shape[2:], cfg.k_cache.dtype)
+    rv = np.zeros((B, ring_slots) + cfg.v_cache.shape[2:], cfg.v_cache.dtype)
+    for s in range(B):
+        st = int(cfg.start[s])
+        for p in range(max(0, st - R0), st):
+            rk[s, p % ring_slots] = cfg.k_cache[s, p % R0]
+            rv[s, p % ring_slots] = cfg.v_cache[s, p % R0]
+    return rk, rv
