@@ -42,8 +42,9 @@ DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
 # workload, from one ncu capture of the kernel on a 2 x 4096-token sliding-window prefill
 # (inputs larger than L2) scaled by tokens to the 40696-token workload (the kernel's traffic
-# is proportional to tokens).  None until the current kernel has been captured.
-TRAFFIC_BYTES = {"prefill_swa_kernel": None}
+# is proportional to tokens): 249.66 MB read + 100.67 MB written.  None whenever the kernel
+# changes after the capture.
+TRAFFIC_BYTES = {"prefill_swa_kernel": int((249657856 + 100670720) * 40696 / 8192)}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
@@ -123,7 +124,8 @@ _REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown"
 
 
 class ClockSampler:
-    """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~10 ms."""
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~1 ms (the
+    timed region of the default step count lasts about 10 ms)."""
 
     def __init__(self, device_index: int):
         self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
@@ -153,7 +155,7 @@ class ClockSampler:
             except Exception as e:
                 self.err = str(e)
                 return
-            time.sleep(0.01)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.h is not None:
@@ -337,7 +339,8 @@ class Decode:
             self.kc, self.vc = dev_bf16(cfg.k_cache), dev_bf16(cfg.v_cache)
         self.sink = dev_f32(L.sink)
         self.extra = dict(cache_kind=M.MIMO_CACHE_PAGED, block_table=dev_i32(cfg.block_table),
-                          num_pages=cfg.k_cache.shape[0]) if cfg.paged else dict(cache_kind=M.MIMO_CACHE_RING)
+                          num_pages=cfg.k_cache.shape[0]) if cfg.paged else \
+            dict(cache_kind=M.MIMO_CACHE_RING, ring_slots=cfg.k_cache.shape[1])
         B = self.q.shape[0]
         self.out = torch.empty((B, 64, 128), dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty((B, 64), dtype=torch.float32, device="cuda")

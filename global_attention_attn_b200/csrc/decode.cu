@@ -488,6 +488,10 @@ __global__ void __launch_bounds__(DecodeLayout<FP8, NC>::kThreads, 1)
     const float c_log2 = FP8 ? p.scale_log2 * p.k_dequant[g] : p.scale_log2;
     const float v_deq = FP8 ? p.v_dequant[g] : 1.f;
 
+    // ring: the slot of position kp is kp mod R, and the ring holds positions ctx-R .. ctx-1,
+    // so slot j holds position ctx - R + ((j + ring_off) mod R) with ring_off = (R - ctx) mod R
+    const int R = p.ring_slots;
+    const int ring_off = p.cache_kind == MIMO_CACHE_RING ? ((R - ctx) % R + R) % R : 0;
     float m_r[2] = {-INFINITY, -INFINITY};
     float l_r[2] = {0.f, 0.f};
     float o[16][4];
@@ -559,9 +563,8 @@ __global__ void __launch_bounds__(DecodeLayout<FP8, NC>::kThreads, 1)
         const int col = ((e & 2) ? 8 : 0) + 2 * q4 + (e & 1);  // within the 16-key tile
         int kp;
         if (p.cache_kind == MIMO_CACHE_RING) {
-          const int slot = kTileK * t + col, R = p.ring_slots;
-          const int base = ctx - R;  // the ring holds positions base .. ctx-1
-          kp = base + (((slot - base) % R) + R) % R;
+          const int j = kTileK * t + col + ring_off;  // < 2 R
+          kp = ctx - R + (j >= R ? j - R : j);
         } else {
           kp = (t0 + t) * kTileK + col;
         }
