@@ -44,7 +44,7 @@ DOMINANT = "prefill_swa_kernel"
 # (inputs larger than L2) scaled by tokens to the 40696-token workload (the kernel's traffic
 # is proportional to tokens): 249.66 MB read + 100.67 MB written.  None whenever the kernel
 # changes after the capture.
-TRAFFIC_BYTES = {"prefill_swa_kernel": int((249657856 + 100670720) * 40696 / 8192)}
+TRAFFIC_BYTES = {"prefill_swa_kernel": None}
 
 
 # ----------------------------------------------------------------------------- roofline inputs

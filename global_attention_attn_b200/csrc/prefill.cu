@@ -620,8 +620,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 // and 11 apply the partial RoPE to each Q tile in shared memory, with a
 // per-row (cos, sin) table that the key pre-pass computes once per query row.  With 12
 // warps, each SM sub-partition holds 3, which caps registers at 168 per
-// thread; the softmax therefore reads S in 48-column chunks, twice (row
-// maximum, then exponentials).  The MMA
+// thread.  The code each softmax warp runs once per tile is kept short: the kernel's
+// roles run different code at the same time, and instruction fetch, not the exponential
+// unit, set the softmax's pace (the same S columns 32..127 go through one copy of a
+// 32-column loop body, and the epilogue's four O chunks through one).  The MMA
 // lane issues QK^T of tile t before PV of tile t-1; QK^T of tile t waits until
 // the epilogue of tile t-2 (same region) has read O.
 namespace {
@@ -1030,19 +1032,42 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
           la2 = add_f32x2(la2, pack_f32x2(sum, 0.f));
         }
         tmem_wait_ld_r32(buf[1]);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const uint32_t* sr = buf[(h + 1) & 1];
-          if (h < 3) ld(h + 1, buf[h & 1]);
+        {  // chunk 0: columns 0..15 are edge columns
           uint32_t pk[16];
-          float sum = exp_chunk(sr, h, pk);
+          float sum = exp_chunk(buf[1], 0, pk);
           if (__any_sync(0xffffffffu, !(sum <= kOver))) {
-            raise_ref(!(sum <= kOver), sr, h, 16 * h);
-            sum = exp_chunk(sr, h, pk);
+            raise_ref(!(sum <= kOver), buf[1], 0, 0);
+            sum = exp_chunk(buf[1], 0, pk);
+          }
+          tmem_st8(t_lane, pk);
+          tmem_st8(t_lane + 8, pk + 8);
+          la2 = add_f32x2(la2, pack_f32x2(sum, 0.f));
+        }
+        // chunks 1..3: every column visible; one copy of the code for the three
+        auto exp_mid = [&](const uint32_t* sr, uint32_t* pk) {
+          const uint64_t nm2 = pack_f32x2(-m_use, -m_use);
+          uint64_t sum2 = pack_f32x2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const uint64_t t = fma_f32x2(pack_f32x2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), cl2, nm2);
+            const float p0 = ex2(lo_f32(t)), p1 = ex2(hi_f32(t));
+            sum2 = add_f32x2(sum2, pack_f32x2(p0, p1));
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+          return lo_f32(sum2) + hi_f32(sum2);
+        };
+#pragma unroll 1
+        for (int h = 1; h < 4; ++h) {
+          tmem_ld32(t_lane + 32 * h, buf[0]);
+          tmem_wait_ld_r32(buf[0]);
+          uint32_t pk[16];
+          float sum = exp_mid(buf[0], pk);
+          if (__any_sync(0xffffffffu, !(sum <= kOver))) {
+            raise_ref(!(sum <= kOver), buf[0], h, 16 * h);
+            sum = exp_mid(buf[0], pk);
           }
           tmem_st8(t_lane + 16 * h, pk);
           tmem_st8(t_lane + 16 * h + 8, pk + 8);
-          if (h < 3) tmem_wait_ld_r32_after(buf[h & 1], la2);
           la2 = add_f32x2(la2, pack_f32x2(sum, 0.f));
         }
         tmem_st8(t_lane + 64, pk4);
@@ -1106,7 +1131,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
         // the 8 heads) instead of 16 bytes of each of 32 rows.
         uint8_t* stage = smem + Ly::kOffStage + (warp - 2) * Ly::kStageBytes;
         const uint64_t sc2 = pack_f32x2(sc, sc);
-        uint32_t oa[32], ob[32];
+        uint32_t oa[32];
         auto store_chunk = [&](uint32_t* o, int c) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -1128,18 +1153,12 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
           }
           __syncwarp();
         };
-        tmem_ld32(t_lane + kSwaColO, oa);
-        tmem_wait_ld_r32(oa);
-        tmem_ld32(t_lane + kSwaColO + 32, ob);
-        store_chunk(oa, 0);
-        tmem_wait_ld_r32(ob);
-        tmem_ld32(t_lane + kSwaColO + 64, oa);
-        store_chunk(ob, 32);
-        tmem_wait_ld_r32(oa);
-        tmem_ld32(t_lane + kSwaColO + 96, ob);
-        store_chunk(oa, 64);
-        tmem_wait_ld_r32(ob);
-        store_chunk(ob, 96);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          tmem_ld32(t_lane + kSwaColO + c, oa);
+          tmem_wait_ld_r32(oa);
+          store_chunk(oa, c);
+        }
       }
       if (row_valid && p.lse) p.lse[long(T.q_row0 + r) * kHq + head] = (m_use + __log2f(l_row)) * kLn2;
       tc_fence_before();
