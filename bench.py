@@ -42,9 +42,9 @@ DOMINANT = "prefill_swa_kernel"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel on the timed
 # workload, from one ncu capture of the kernel on a 2 x 4096-token sliding-window prefill
 # (inputs larger than L2) scaled by tokens to the 40696-token workload (the kernel's traffic
-# is proportional to tokens): 249.66 MB read + 100.67 MB written.  None whenever the kernel
+# is proportional to tokens): 249.64 MB read + 101.57 MB written.  None whenever the kernel
 # changes after the capture.
-TRAFFIC_BYTES = {"prefill_swa_kernel": None}
+TRAFFIC_BYTES = {"prefill_swa_kernel": int((249644800 + 101571328) * 40696 / 8192)}
 
 
 # ----------------------------------------------------------------------------- roofline inputs
