@@ -58,6 +58,9 @@ int check_layer(const char* fn, const mimo_layer& L) {
   return MIMO_OK;
 }
 
+// Every bounded wait of the kernels gives up after this long by default.
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
 RopeFreqs make_freqs(double base) {
   RopeFreqs f;
   for (int j = 0; j < kHalf; ++j) f.inv_freq[j] = std::pow(base, -2.0 * double(j) / double(kRope));
@@ -220,6 +223,95 @@ size_t decode_workspace(int batch, int q_len, int max_seq_len, int window) {
   return round256(rows * kHq * ns * kDv * 4) + round256(rows * kHq * ns * 2 * 4);
 }
 
+// Draft verification of a global layer on a bf16 paged cache: the q_len rows of a sequence's 16
+// heads fill half or all of the tensor-core prefill kernel's 128-row tile, which reads each
+// 128-key page once per split for all of them.  Splits are whole pages: the decode's split length
+// (a multiple of 128), doubled beyond 8192 keys, where a unit's fixed costs (its query tile, the
+// partials written and merged) weigh more than the balance of the last round; never shorter than
+// the decode's, so the partials fit its workspace and its combine pass merges them.
+int decode_drafts_paged_tc(const char* fn, const mimo_decode_args* a, int q_len, void* stream) {
+  DevState d;
+  if (int rc = dev_state(fn, &d)) return rc;
+  EncodeTiledFn enc;
+  if (int rc = get_encoder(fn, &enc)) return rc;
+  const int hkv = a->layer.num_kv_heads;
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  const long rows = long(a->num_pages) * kPage;
+  int rc = make_map(fn, enc, &p.tm_q, a->q, long(a->batch) * q_len, kHq, kDqk, 16, prefill_rows_per_tile(1));
+  if (!rc) rc = make_map(fn, enc, &p.tm_k0, a->k_cache, rows, hkv, kDqk, 1, 128);
+  if (!rc) rc = make_map(fn, enc, &p.tm_k12, a->k_cache, rows, hkv, kDqk, 1, 128);
+  if (!rc) rc = make_map(fn, enc, &p.tm_v, a->v_cache, rows, hkv, kDv, 1, 128);
+  if (rc) return rc;
+  const int split_len = decode_split_len(a->max_seq_len) * (a->max_seq_len > 8192 ? 2 : 1);
+  const int max_splits = (a->max_seq_len + split_len - 1) / split_len;
+  p.num_seqs = a->batch;
+  p.total_q = a->batch * q_len;
+  p.hkv = hkv;
+  p.mode = kModePaged;
+  p.window = 0;
+  p.max_pages = a->max_pages;
+  p.num_pages = a->num_pages;
+  p.scale_log2 = a->layer.softmax_scale * 1.4426950408889634f;
+  p.v_scale = a->layer.v_scale;
+  p.sink = a->layer.sink;
+  p.out = static_cast<uint16_t*>(a->out);
+  p.lse = a->lse;
+  p.rope = make_freqs(a->layer.rope_base);
+  p.status = d.status;
+  p.wait_ns = kWaitNs;
+  p.uq = q_len;
+  if (max_splits > 1) {
+    p.split_tiles = split_len / kPage;
+    p.max_splits = max_splits;
+    p.ws_o = static_cast<float*>(a->workspace);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(a->workspace) +
+                                       round256(size_t(a->batch) * q_len * kHq * max_splits * kDv * 4));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long work = long(a->batch) * hkv * max_splits;
+  const int grid = int(work < d.sms ? work : d.sms);
+  if (a->ev_kernel_begin) {
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_kernel_begin), st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: ev_kernel_begin: %s", fn, cudaGetErrorString(e));
+  }
+  for (int s0 = 0; s0 < a->batch; s0 += kPrefillMaxSeqsPerLaunch) {
+    PrefillParams q = p;
+    q.seq_base = s0;
+    q.num_seqs = a->batch - s0 < kPrefillMaxSeqsPerLaunch ? a->batch - s0 : kPrefillMaxSeqsPerLaunch;
+    q.seq_lens = a->seq_lens + s0;
+    q.block_table = a->block_table + long(s0) * a->max_pages;
+    cudaError_t e = launch_prefill(q, 1, grid, st, false);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  if (a->ev_kernel_end) {
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_kernel_end), st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: ev_kernel_end: %s", fn, cudaGetErrorString(e));
+  }
+  if (max_splits > 1) {
+    DecodeParams c;
+    std::memset(&c, 0, sizeof(c));
+    c.batch = a->batch;
+    c.hkv = hkv;
+    c.group = kHq / hkv;
+    c.q_len = q_len;
+    c.window = 0;
+    c.split_len = split_len;
+    c.max_splits = max_splits;
+    c.v_scale = a->layer.v_scale;
+    c.sink = a->layer.sink;
+    c.seq_lens = a->seq_lens;
+    c.out = p.out;
+    c.lse = a->lse;
+    c.ws_o = p.ws_o;
+    c.ws_ml = p.ws_ml;
+    c.status = d.status;
+    cudaError_t e = launch_decode_combine(c, st);
+    if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: combine launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  return MIMO_OK;
+}
+
 }  // namespace
 }  // namespace mimo
 
@@ -362,6 +454,9 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
                   a->workspace ? a->workspace_bytes : size_t(0));
     if (!aligned16(a->workspace)) return fail(MIMO_ERR_INVALID_ARG, "%s: workspace is not 16-byte aligned", fn);
   }
+  if (q_len >= 2 && a->cache_kind == MIMO_CACHE_PAGED && a->cache_dtype != MIMO_DTYPE_FP8_E4M3 &&
+      a->layer.window <= 0 && a->layer.num_kv_heads == 4)
+    return decode_drafts_paged_tc(fn, a, q_len, stream);
   DevState d;
   if (int rc = dev_state(fn, &d)) return rc;
   EncodeTiledFn enc;
@@ -426,8 +521,6 @@ int mimo_attn_decode(const mimo_decode_args* a, void* stream) {
 namespace mimo {
 namespace {
 
-// Every bounded wait of the kernels gives up after this long by default.
-constexpr unsigned long long kWaitNs = 2000000000ull;
 
 int prefill_impl(const char* fn, const mimo_prefill_args* a, void* stream, unsigned long long wait_ns,
                  int withhold_q) {

@@ -790,6 +790,10 @@ cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* 
   if (e != cudaSuccess) return e;
   if (ev_end && (e = cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s)) != cudaSuccess) return e;
   if (p.max_splits <= 1) return e;
+  return launch_decode_combine(p, s);
+}
+
+cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t s) {
   const long warps = long(p.batch) * p.q_len * kHq;
   decode_combine_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, s>>>(p);
   return cudaGetLastError();

@@ -107,6 +107,17 @@ struct PrefillParams {
   unsigned* status;
   unsigned long long wait_ns;  // limit of every bounded wait in the kernel
   int withhold_q;              // failure-detection test: the producer never loads a query tile
+  // Draft verification on a paged cache (global kernel only): with cu_q null, sequence s holds
+  // the uq query rows (seq_base + s) * uq + i at positions seq_lens[s] - uq + i, i < uq <= 8.
+  int uq;
+  const int32_t* seq_lens;
+  // Split-KV (with uq): split i of a sequence takes key tiles [i * split_tiles, (i + 1) *
+  // split_tiles); each split writes its unnormalised O and (running max in log2 units, sum)
+  // to ws_o [rows, 64, max_splits, 128] / ws_ml [rows, 64, max_splits, 2] for the decode's
+  // combine pass, which adds the sink.  split_tiles 0: one split, final rows written.
+  int split_tiles, max_splits;
+  float* ws_o;
+  float* ws_ml;
 };
 
 // Pre-pass of the prefill: rotated key copies into the workspace.
@@ -133,6 +144,8 @@ struct RopeKParams {
 cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s);
 // ev_begin / ev_end: optional cudaEvent_t recorded around the decode kernel (not the combine)
 cudaError_t launch_decode(const DecodeParams& p, int sms, cudaStream_t s, void* ev_begin, void* ev_end);
+// The combine pass alone: merges p.max_splits partials per (query row, head) of ws_o / ws_ml.
+cudaError_t launch_decode_combine(const DecodeParams& p, cudaStream_t s);
 // Row blocks of a decode unit (q_len rows of `group` heads), consumer warps per producer and
 // row parts per unit.
 void decode_rows(int q_len, int group, int* n_blocks, int* nc, int* n_rp);

@@ -88,6 +88,7 @@ struct TileInfo {
   int key_lo;                // first key position that exists
   int krow_base, kpos_base;  // contiguous key sources: row of position kpos_base
   int new_row0, new_pos0;    // ring-cache chunk: row of the first new key in k / v, its position
+  int split;                 // split-KV: the tile's split (key tiles from split * split_tiles), else -1
 };
 
 // Per-CTA copy of the per-sequence quantities the roles need for every tile.
@@ -116,13 +117,37 @@ __device__ __forceinline__ void fill_seq_table(const PrefillParams& p, const Seq
     const int s = s0 + lane;
     int n = 0;
     if (s < p.num_seqs) {
-      const int q0 = p.cu_q[s], ql = p.cu_q[s + 1] - q0;
-      n = (ql + R - 1) / R;
-      S.q0[s] = q0;
-      S.qlen[s] = ql;
-      S.clen[s] = p.cache_lens ? p.cache_lens[s] : 0;
-      S.k0[s] = p.cu_k ? p.cu_k[s] : 0;
-      S.klen[s] = p.cu_k ? p.cu_k[s + 1] - p.cu_k[s] : 0;
+      if (KIND == 1 && p.uq > 0) {
+        // uq rows (uq <= R: one M tile) ending at the context's last position; with split-KV
+        // one work item per split of the context's keys
+        const int ql = p.uq, ctx = p.seq_lens[s];
+        n = 1;
+        if (p.split_tiles > 0) {
+          const int len = p.split_tiles * 128;
+          n = ctx > 0 ? (ctx - 1) / len + 1 : 0;
+          if (n > p.max_splits) {  // a context beyond max_seq_len: its extra keys are not attended
+            atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
+            n = p.max_splits;
+          }
+        }
+        if (ctx < ql) {  // fewer positions than query rows: nothing to attend
+          atomicOr(p.status, MIMO_STATUS_BAD_INDEX);
+          n = 0;
+        }
+        S.q0[s] = (p.seq_base + s) * ql;
+        S.qlen[s] = ql;
+        S.clen[s] = ctx;  // as for a paged prefill: every key, the drafts included, is in the cache
+        S.k0[s] = 0;
+        S.klen[s] = 0;
+      } else {
+        const int q0 = p.cu_q[s], ql = p.cu_q[s + 1] - q0;
+        n = (ql + R - 1) / R;
+        S.q0[s] = q0;
+        S.qlen[s] = ql;
+        S.clen[s] = p.cache_lens ? p.cache_lens[s] : 0;
+        S.k0[s] = p.cu_k ? p.cu_k[s] : 0;
+        S.klen[s] = p.cu_k ? p.cu_k[s + 1] - p.cu_k[s] : 0;
+      }
     }
     int incl = n;
 #pragma unroll
@@ -144,7 +169,7 @@ __device__ __forceinline__ bool locate(const PrefillParams& p, const SeqTable& S
   constexpr int R = Cfg<KIND>::R;
   const int total = S.tile_start[p.num_seqs] * p.hkv;
   if (w >= total) return false;
-  if (KIND == 1) {
+  if (KIND != 0) {
     // CTA i takes items i, i + grid, ...: reverse every other round of grid items, so the
     // CTA that gets a round's longest tile gets the next round's shortest
     const int G = int(gridDim.x), round = w / G, base = round * G;
@@ -159,7 +184,14 @@ __device__ __forceinline__ bool locate(const PrefillParams& p, const SeqTable& S
   T.s = lo;
   T.ntiles = S.tile_start[lo + 1] - S.tile_start[lo];
   int t = tt - S.tile_start[lo];
-  if (KIND == 1) t = T.ntiles - 1 - t;
+  T.split = -1;
+  if (KIND == 1 && p.split_tiles > 0) {  // items of a sequence are the splits of its one M tile
+    T.split = t;
+    T.ntiles = 1;
+    t = 0;
+  } else if (KIND != 0) {
+    t = T.ntiles - 1 - t;
+  }
   T.t = t;
   T.g = w % p.hkv;
   const int qlen = S.qlen[lo], clen = S.clen[lo];
@@ -196,6 +228,12 @@ __device__ __forceinline__ void key_tiles(const PrefillParams& p, const TileInfo
     const int lo = p.window > 0 ? max(0, T.qpos0 - p.window + 1) : 0;
     *j_lo = max(lo, 0) / 128;
     *n = max(qlast, 0) / 128 - *j_lo + 1;
+    if (T.split >= 0) {  // this split's share; at least one tile (its keys are masked if none is visible)
+      const int a = T.split * p.split_tiles;
+      const int e = min(*j_lo + *n, a + p.split_tiles);
+      *j_lo = max(*j_lo, a);
+      *n = max(e - *j_lo, 1);
+    }
   }
 }
 template <int KIND>
@@ -482,8 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const bool row_valid = r < T.rows_valid;
       const int qp = T.qpos0 + r;
       const int head = T.g * G + hq;
-      float m_run = sink_l2[head];
-      float l_run = p.sink ? 1.f : 0.f;
+      // a split's partial leaves the sink to the combine pass
+      float m_run = T.split >= 0 ? -INFINITY : sink_l2[head];
+      float l_run = (p.sink && T.split < 0) ? 1.f : 0.f;
       // visible key positions of this row: [vis_lo, vis_hi]
       const int vis_hi = row_valid ? qp : -0x40000000;
       const int vis_lo = max(T.key_lo, p.window > 0 ? qp - p.window + 1 : -0x40000000);
@@ -575,6 +614,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       if (nkv >= 2 && !(ok = wait_w(pv_done, (jj - 2) & 1))) break;
       if (!(ok = wait_w(pv_done, (jj - 1) & 1))) break;
       tc_fence_after();
+      if (T.split >= 0) {
+        // split-KV partial: O as accumulated (relative to m_run), with (m_run, l_run)
+        const long pr = (long(T.q_row0 + r) * kHq + head) * p.max_splits + T.split;
+        float* dst = p.ws_o + pr * kDv;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + kColO + c, o);
+          tmem_wait_ld_r32(o);
+          if (row_valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+        }
+        if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + 2 * pr) = make_float2(m_run, l_run);
+        tc_fence_before();
+        mbar_arrive(o_empty);
+        ++mt;
+        T = Tn;
+        have = have_next;
+        continue;
+      }
       const float sc = p.v_scale / l_run;
       uint16_t* orow = p.out + (long(T.q_row0 + r) * kHq + head) * kDv;
 #pragma unroll
@@ -1385,7 +1447,7 @@ cudaError_t launch_rope_k(const RopeKParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-int prefill_rows_per_tile(int kind) { return kind == 0 ? Cfg<0>::R : Cfg<1>::R; }
+int prefill_rows_per_tile(int kind) { return kind == 0 ? Cfg<0>::R : Cfg<1>::R; }  // query rows of one TMA box
 int prefill_key_tile(int kind) { return kind == 0 ? Cfg<0>::BN : Cfg<1>::BN; }
 
 cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStream_t s, bool pdl) {

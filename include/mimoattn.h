@@ -218,6 +218,16 @@ MIMO_API int mimo_attn_prefill_stall_test(const mimo_prefill_args* args, void* s
  * Layouts: q [batch * q_len, 64, 192] bf16 pre-RoPE; out [batch * q_len, 64, 128] bf16;
  * lse [batch * q_len, 64] fp32 or NULL.  max_seq_len is a host-side upper bound of
  * seq_lens (it sizes the split-KV grid and the workspace); every seq_lens[s] >= q_len.
+ * A sequence whose seq_lens is below q_len sets MIMO_STATUS_BAD_INDEX; its rows are
+ * undefined.  A seq_lens above max_seq_len breaks the contract: keys beyond the splits
+ * that max_seq_len sizes are not attended (reported as MIMO_STATUS_BAD_INDEX whenever the
+ * call has more than one split).
+ *
+ * Kernels: one token per sequence, a ring cache, an E4M3 cache or a window run the
+ * split-KV decode kernel; draft rows (q_len >= 2) of a global layer (4 KV heads, no
+ * window) on a bf16 paged cache run the tensor-core prefill kernel, whose 128-row tile
+ * holds the q_len x 16 query rows of one KV head, over page-aligned splits, then the same
+ * combine pass.  Either way the split-KV workspace is the one the size queries give.
  */
 #define MIMO_MAX_DRAFTS 8
 typedef struct {

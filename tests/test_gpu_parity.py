@@ -528,6 +528,71 @@ def test_decode_drafts_split_edges_and_window():
     parity(out, lse, *oracle.decode(cfg), "drafts, paged window 1000 with sink")
 
 
+def _global_drafts(seed, ctx, q_len, sink=False):
+    """A global-layer paged cache over contexts `ctx` scored by q_len draft rows per sequence."""
+    import dataclasses
+    bt, pool = configs.paged_layout(seed, 1, ctx)
+    gl = configs.Decode(configs.global_layer(), None, ctx, configs.cached_keys(seed, 2, (pool, 128, 4, 192)),
+                        configs.bf16_normal(seed, 3, (pool, 128, 4, 128)), block_table=bt,
+                        name=f"global_drafts_{len(ctx)}")
+    if sink:
+        gl.layer = dataclasses.replace(gl.layer, sink=synth.normal_f32(synth.stream_seed(seed, 9), (64,)))
+    return configs.with_drafts(gl, q_len, seed=seed + 1)
+
+
+@pytest.mark.parametrize("q_len", [2, 4, 8])
+def test_decode_drafts_global_tensor_core(q_len):
+    """Draft rows of a global layer on a bf16 paged cache go through the tensor-core kernel
+    (the q_len x 16 rows of a KV head in one 128-row tile) with page-aligned splits and the
+    decode's combine pass: contexts that end just before, at and after a split boundary, a
+    sink (the combine adds it once), and a batch whose longest context needs one split only
+    (no workspace, final rows written by the kernel itself)."""
+    ctx = np.array([q_len, q_len + 1, 127, 128, 129, 511, 512, 513, 512 + q_len - 1, 1024 + q_len, 2047, 3001],
+                   np.int32)
+    for sink in (False, True):
+        cfg = _global_drafts(760 + q_len, ctx, q_len, sink)
+        out, lse = decode_cfg(cfg)
+        parity(out, lse, *oracle.decode(cfg), f"{cfg.name} sink={sink}")
+    cfg = _global_drafts(765 + q_len, np.array([q_len, 100, 200, 256], np.int32), q_len, True)
+    out, lse = decode_cfg(cfg)
+    parity(out, lse, *oracle.decode(cfg), f"{cfg.name}: one split")
+
+
+def test_decode_drafts_global_more_sequences_than_one_launch():
+    """300 sequences: the tensor-core path launches per group of 256 sequences; rows of the
+    second launch keep their global row numbers in the partials and the output."""
+    ctx = synth.randint(synth.stream_seed(770, 0), 300, 2, 1400).astype(np.int32)
+    cfg = _global_drafts(771, ctx, 2)
+    out, lse = decode_cfg(cfg)
+    sel = np.array([0, 1, 2, 127, 254, 255, 256, 257, 298, 299], np.int32)
+    ro, rl = oracle.decode(cfg, seqs=sel)
+    import torch
+    rows = torch.as_tensor(np.repeat(sel, 2) * 2 + np.tile([0, 1], len(sel)), device=out.device)
+    parity(out[rows], lse[rows], ro, rl, "300 sequences x 2 drafts")
+
+
+def test_decode_kernels_by_route():
+    """Which kernels a decode call launches: draft rows of a global layer on a bf16 paged cache
+    run the tensor-core prefill kernel and the combine pass, not the decode kernel; one token
+    per sequence runs the decode kernel."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    cfg = _global_drafts(780, np.array([700, 3000, 5000], np.int32), 4)
+    one = configs.with_drafts(cfg, 1, seed=781)
+    decode_cfg(cfg)
+    decode_cfg(one)
+    torch.cuda.synchronize()
+    names = []
+    for c in (cfg, one):
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            decode_cfg(c)
+            torch.cuda.synchronize()
+        names.append(" ".join(e.name for e in prof.events() if "mimo" in e.name))
+    assert "prefill_kernel" in names[0] and "decode_combine_kernel" in names[0], names[0]
+    assert "decode_kernel<" not in names[0], names[0]
+    assert "decode_kernel<" in names[1] and "prefill_kernel" not in names[1], names[1]
+
+
 @pytest.mark.parametrize("ring", [False, True])
 def test_decode_drafts_fp8(ring):
     import dataclasses

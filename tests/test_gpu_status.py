@@ -140,3 +140,24 @@ def test_fp8_append_skips_and_reports_bad_scales():
     assert not kb[0, :n, 1:3].any() and not vb[0, :n, 1:3].any()   # heads 1 and 2 skipped
     assert kb[0, :n, 0].any() and kb[0, :n, 3].any()               # heads 0 and 3 written
     assert not kb[0, n:].any()
+
+
+def test_draft_rows_beyond_a_short_context_are_reported():
+    """A context shorter than the draft rows (seq_lens below q_len) on the tensor-core draft path:
+    reported as MIMO_STATUS_BAD_INDEX, nothing attended for it; the other sequences unaffected."""
+    import torch
+    import global_attention_attn_b200 as M
+    _, gl = configs.decode_batch(seed=943, B=5, ctx_range=(600, 3000))
+    cfg = configs.with_drafts(gl, 4, seed=944)
+    ctx = cfg.ctx.copy()
+    ctx[3] = 2
+    L = cfg.layer
+    out, lse = M.mimo_attn_decode(dev_bf16(cfg.q), dev_i32(ctx), max_seq_len=int(ctx.max()),
+                                  num_kv_heads=4, rope_base=L.rope_base, window=0, k_cache=dev_bf16(cfg.k_cache),
+                                  v_cache=dev_bf16(cfg.v_cache), cache_kind=M.MIMO_CACHE_PAGED,
+                                  block_table=dev_i32(cfg.block_table), num_pages=cfg.k_cache.shape[0], q_len=4)
+    assert poll()[1] == M.MIMO_STATUS_BAD_INDEX
+    good = np.array([0, 1, 2, 4])
+    ro, rl = oracle.decode(cfg, seqs=good)
+    idx = torch.as_tensor(np.repeat(good, 4) * 4 + np.tile(np.arange(4), len(good)), device=out.device)
+    parity(out[idx], lse[idx], ro, rl, "drafts, other sequences of a batch with a too-short context")
