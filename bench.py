@@ -267,7 +267,8 @@ class HostPipeline:
     on the caller's stream: the inputs of later sequences travel host -> device on one copy
     stream while a sequence computes, and the outputs of earlier ones travel back on another
     (PCIe carries both directions at once).  Every step copies all of its inputs in and
-    all of its outputs out."""
+    all of its outputs out.  Sequences go longest first, so the output copy left after the
+    last call (the step's tail) is the shortest one."""
 
     def __init__(self, step):
         import torch
@@ -281,6 +282,7 @@ class HostPipeline:
         self.out_h = torch.empty_like(step.out, device="cpu").pin_memory()
         self.lse_h = torch.empty_like(step.lse, device="cpu").pin_memory()
         lens = np.diff(np.asarray(self.cu))
+        self.order = [int(i) for i in np.argsort(-lens, kind="stable")]
         self.cu1_h = [pin(torch.tensor([0, int(n)], dtype=torch.int32)) for n in lens]
         self.cu1_d = [torch.empty(2, dtype=torch.int32, device="cuda") for _ in lens]
         self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -296,10 +298,10 @@ class HostPipeline:
         cur = torch.cuda.current_stream()
         self.s_in.wait_stream(cur)   # the previous step's calls and copies are done
         self.s_out.wait_stream(cur)
-        arrived = []
+        arrived = {}
         with torch.cuda.stream(self.s_in):
             st.sink.copy_(self.s_h, non_blocking=True)
-            for s in range(len(cu) - 1):
+            for s in self.order:
                 a, b = cu[s], cu[s + 1]
                 st.q[a:b].copy_(self.q_h[a:b], non_blocking=True)
                 st.k[a:b].copy_(self.k_h[a:b], non_blocking=True)
@@ -307,8 +309,8 @@ class HostPipeline:
                 self.cu1_d[s].copy_(self.cu1_h[s], non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(self.s_in)
-                arrived.append(ev)
-        for s in range(len(cu) - 1):
+                arrived[s] = ev
+        for s in self.order:
             a, b = cu[s], cu[s + 1]
             cur.wait_event(arrived[s])
             M.mimo_attn_prefill(st.q[a:b], st.k[a:b], st.v[a:b], self.cu1_d[s], self.cu1_d[s],

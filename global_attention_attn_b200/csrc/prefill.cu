@@ -243,7 +243,9 @@ __device__ __forceinline__ int key_tile_start(const TileInfo& T, int j) {
 
 }  // namespace
 
-template <int KIND>
+// SPLIT: the draft-row mode's split-KV partials (p.split_tiles > 0); a separate instance, so
+// the prefill's own code carries none of it
+template <int KIND, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
   using C = Cfg<KIND>;
   using Ly = Layout<KIND>;
@@ -521,8 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int qp = T.qpos0 + r;
       const int head = T.g * G + hq;
       // a split's partial leaves the sink to the combine pass
-      float m_run = T.split >= 0 ? -INFINITY : sink_l2[head];
-      float l_run = (p.sink && T.split < 0) ? 1.f : 0.f;
+      float m_run = SPLIT ? -INFINITY : sink_l2[head];
+      float l_run = (p.sink && !SPLIT) ? 1.f : 0.f;
       // visible key positions of this row: [vis_lo, vis_hi]
       const int vis_hi = row_valid ? qp : -0x40000000;
       const int vis_lo = max(T.key_lo, p.window > 0 ? qp - p.window + 1 : -0x40000000);
@@ -614,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       if (nkv >= 2 && !(ok = wait_w(pv_done, (jj - 2) & 1))) break;
       if (!(ok = wait_w(pv_done, (jj - 1) & 1))) break;
       tc_fence_after();
-      if (T.split >= 0) {
+      if constexpr (SPLIT) {
         // split-KV partial: O as accumulated (relative to m_run), with (m_run, l_run)
         const long pr = (long(T.q_row0 + r) * kHq + head) * p.max_splits + T.split;
         float* dst = p.ws_o + pr * kDv;
@@ -1468,12 +1470,12 @@ cudaError_t launch_prefill(const PrefillParams& p, int kind, int grid, cudaStrea
     cfg.dynamicSmemBytes = SwaLayout::kAlloc;
     return cudaLaunchKernelEx(&cfg, prefill_swa_kernel, p);
   }
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Layout<1>::kAlloc);
+  auto* fn = p.split_tiles > 0 ? prefill_kernel<1, true> : prefill_kernel<1, false>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<1>::kAlloc);
   if (e != cudaSuccess) return e;
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Layout<1>::kAlloc;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<1>, p);
+  return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
 }  // namespace mimo

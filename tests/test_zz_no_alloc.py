@@ -7,6 +7,7 @@ This file is collected last on purpose: if it fails, a run that stops at the fir
 failure has already run every other test.
 """
 import ctypes as C
+import gc
 
 import numpy as np
 import pytest
@@ -69,12 +70,21 @@ def test_noalloc_decode_matches_decode_on_two_calls(cuda_ok):
         B = t["q"].shape[0]
         out = torch.empty((B, 64, 128), dtype=torch.bfloat16, device="cuda")
         lse = torch.empty((B, 64), dtype=torch.float32, device="cuda")
-        torch.cuda.synchronize()
-        before, free_before = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
-        M.mimo_attn_decode_noalloc(t["q"], t["ctx"], out=out, lse=lse, **_kw(t))
-        torch.cuda.synchronize()
-        assert torch.cuda.memory_allocated() == before
-        assert torch.cuda.mem_get_info()[0] == free_before
+        kw = _kw(t)  # its device tensors exist before the measurement
+        # no garbage collection inside the measured window: a collection there frees
+        # earlier tensors and moves torch's count without the call having done anything
+        gc.collect()
+        gc.disable()
+        try:
+            torch.cuda.synchronize()
+            before, free_before = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+            M.mimo_attn_decode_noalloc(t["q"], t["ctx"], out=out, lse=lse, **kw)
+            torch.cuda.synchronize()
+            after, free_after = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+        finally:
+            gc.enable()
+        assert after == before
+        assert free_after == free_before
         outs.append((out, lse))
     for t, (ro, rl), (o, l) in zip(cases, refs, outs):
         d = (o.float() - ro.float()).abs()
