@@ -492,6 +492,10 @@ __global__ void __launch_bounds__(DecodeLayout<FP8, NC>::kThreads, 1)
     // so slot j holds position ctx - R + ((j + ring_off) mod R) with ring_off = (R - ctx) mod R
     const int R = p.ring_slots;
     const int ring_off = p.cache_kind == MIMO_CACHE_RING ? ((R - ctx) % R + R) % R : 0;
+    // a paged tile whose keys every row of the block sees needs no mask: [lo_all, hi_all] is the
+    // key range all of the block's rows see (empty when a row is padding)
+    const int lo_all = __reduce_max_sync(0xffffffffu, max(lo_r[0], lo_r[1]));
+    const int hi_all = __reduce_min_sync(0xffffffffu, min(hi_r[0], hi_r[1]));
     float m_r[2] = {-INFINITY, -INFINITY};
     float l_r[2] = {0.f, 0.f};
     float o[16][4];
@@ -558,8 +562,10 @@ __global__ void __launch_bounds__(DecodeLayout<FP8, NC>::kThreads, 1)
         s1[i] = acc[2][i] + acc[3][i];
       }
       // positions of this thread's four key columns, visible or not to each of its two rows
+      const bool interior = p.cache_kind == MIMO_CACHE_PAGED && (t0 + t) * kTileK >= lo_all &&
+                            (t0 + t) * kTileK + kTileK - 1 <= hi_all;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < 4 && !interior; ++e) {
         const int col = ((e & 2) ? 8 : 0) + 2 * q4 + (e & 1);  // within the 16-key tile
         int kp;
         if (p.cache_kind == MIMO_CACHE_RING) {
