@@ -1239,14 +1239,28 @@ __global__ void __launch_bounds__(kSwaThreads, 1) prefill_swa_kernel(const __gri
 }
 
 // ---------------------------------------------------------------- key pre-pass
-// Position of query row `row` (its sequence found by bisection of cu_q): the queries of a
-// sequence are the last q_len of its ctx = cached + new keys.
-__device__ __forceinline__ int query_position(const RopeKParams& p, long row) {
-  int lo = 0, hi = p.num_seqs;
+// Largest s in [0, n) with off(s) <= x (off non-decreasing), for a whole warp that passes
+// the same x: up to 32 sequences with one load per lane and a ballot (one memory round
+// trip, where a bisection takes log2 n dependent ones), else by bisection.
+template <typename F>
+__device__ __forceinline__ int warp_find_seq(int n, long x, F off) {
+  if (n <= 32) {
+    const int lane = threadIdx.x & 31;
+    const unsigned m = __ballot_sync(0xffffffffu, lane < n && off(lane) <= x);
+    return m ? 31 - __clz(m) : 0;
+  }
+  int lo = 0, hi = n;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (p.cu_q[mid] <= row) lo = mid; else hi = mid;
+    if (off(mid) <= x) lo = mid; else hi = mid;
   }
+  return lo;
+}
+
+// Position of query row `row` (warp-collective): the queries of a sequence are the last
+// q_len of its ctx = cached + new keys.
+__device__ __forceinline__ int query_position(const RopeKParams& p, long row) {
+  const int lo = warp_find_seq(p.num_seqs, row, [&](int i) { return long(p.cu_q[i]); });
   const int qlen = p.cu_q[lo + 1] - p.cu_q[lo];
   const int ctx = (p.cache_lens ? p.cache_lens[lo] : 0) + (p.cu_k[lo + 1] - p.cu_k[lo]);
   return ctx - qlen + int(row - p.cu_q[lo]);
@@ -1279,11 +1293,8 @@ __global__ void __launch_bounds__(256) rope_k_contig_kernel(const RopeKParams p)
       a = __ldg(src);
       b = __ldg(src + 4);
     }
-    int lo = 0, hi = p.num_seqs;  // find s with cu_k[s] <= row < cu_k[s+1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.cu_k[mid] <= row) lo = mid; else hi = mid;
-    }
+    // s with cu_k[s] <= row < cu_k[s+1]
+    const int lo = warp_find_seq(p.num_seqs, row, [&](int i) { return long(p.cu_k[i]); });
     pos_k = (p.cache_lens ? p.cache_lens[lo] : 0) + int(row - p.cu_k[lo]);
     rope_cos_sin(pos_k, p.rope.inv_freq[lane], &c_j, &s_j);
     float2 cs[8];
@@ -1332,11 +1343,8 @@ __global__ void __launch_bounds__(256) rope_k_ext_kernel(const RopeKParams p) {
   float c_j = 0.f, s_j = 0.f;
   if (key_row) {
     const int e = int(wid);
-    int lo = 0, hi = p.num_seqs;  // ext start of s: cu_k[s] + 128 s
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.cu_k[mid] + 128 * mid <= e) lo = mid; else hi = mid;
-    }
+    // the sequence whose ext rows (its 128 halo rows, then its new rows) hold row e
+    const int lo = warp_find_seq(p.num_seqs, e, [&](int i) { return long(p.cu_k[i]) + 128L * i; });
     const int s = lo, i = e - (p.cu_k[s] + 128 * s);
     const int clen = p.cache_lens ? p.cache_lens[s] : 0;
     uint4* kd = reinterpret_cast<uint4*>(p.ws_k + long(e) * HKV * kDqk);
