@@ -125,7 +125,7 @@ _REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown"
 
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~1 ms (the
-    timed region of the default step count lasts about 10 ms)."""
+    timed region of the default step count lasts about 10 ms), in a thread."""
 
     def __init__(self, device_index: int):
         self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
@@ -158,6 +158,10 @@ class ClockSampler:
             time.sleep(0.001)
 
     def __enter__(self):
+        # the launching thread holds the interpreter lock between calls; hand it over every
+        # 0.1 ms (the default is 5 ms) so that the sampler runs during a ~10 ms timed region
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(1e-4)
         if self.h is not None:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
@@ -167,6 +171,7 @@ class ClockSampler:
         self._stop.set()
         if self.h is not None:
             self.t.join()
+        sys.setswitchinterval(self._switch)
 
     def summary(self):
         d = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
