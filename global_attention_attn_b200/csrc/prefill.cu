@@ -620,16 +620,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         // split-KV partial: O as accumulated (relative to m_run), with (m_run, l_run)
         const long pr = (long(T.q_row0 + r) * kHq + head) * p.max_splits + T.split;
         float* dst = p.ws_o + pr * kDv;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(t_lane + kColO + c, o);
-          tmem_wait_ld_r32(o);
-          if (row_valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+        // the whole row of O in one load round trip
+        uint32_t o[128];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-          }
+        for (int c = 0; c < 128; c += 32) tmem_ld32(t_lane + kColO + c, o + c);
+        tmem_wait_ld_r64(o);
+        tmem_wait_ld_r64(o + 64);
+        if (row_valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) d4[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
         if (row_valid) *reinterpret_cast<float2*>(p.ws_ml + 2 * pr) = make_float2(m_run, l_run);
         tc_fence_before();
@@ -641,11 +641,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       }
       const float sc = p.v_scale / l_run;
       uint16_t* orow = p.out + (long(T.q_row0 + r) * kHq + head) * kDv;
+      // the whole row of O in one load round trip
+      uint32_t oall[128];
+#pragma unroll
+      for (int c = 0; c < 128; c += 32) tmem_ld32(t_lane + kColO + c, oall + c);
+      tmem_wait_ld_r64(oall);
+      tmem_wait_ld_r64(oall + 64);
 #pragma unroll
       for (int c = 0; c < 128; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(t_lane + kColO + c, o);
-        tmem_wait_ld_r32(o);
+        const uint32_t* o = oall + c;
         uint4 pk[4];
         uint32_t* w32 = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
