@@ -124,7 +124,7 @@ _REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown"
 
 
 class ClockSampler:
-    """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~1 ms (the
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML every ~0.2 ms (the
     timed region of the default step count lasts about 10 ms), in a thread."""
 
     def __init__(self, device_index: int):
@@ -155,7 +155,7 @@ class ClockSampler:
             except Exception as e:
                 self.err = str(e)
                 return
-            time.sleep(0.001)
+            time.sleep(0.0002)
 
     def __enter__(self):
         # the launching thread holds the interpreter lock between calls; hand it over every
