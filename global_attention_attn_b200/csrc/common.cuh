@@ -124,16 +124,5 @@ __device__ __forceinline__ void rope_chunk_pair_cs4(uint4& lo, uint4& hi, const 
   }
 }
 
-// Same angle, reduced in float64, with the MUFU sine / cosine of the reduced
-// float32 angle (absolute error ~1e-6 on [-pi, pi], far below the fp16 rounding
-// of the rotated values).  For per-tile tables where the accurate sincosf costs
-// more than the whole rotation.
-__device__ __forceinline__ void rope_cos_sin_fast(int pos, double inv_freq, float* c, float* s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double theta = double(pos) * inv_freq;
-  const double k = rint(theta * (1.0 / two_pi));
-  const float r = float(fma(-k, two_pi, theta));
-  __sincosf(r, s, c);
-}
 
 }  // namespace mimo
