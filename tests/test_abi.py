@@ -160,6 +160,13 @@ def _decode_args(**over):
     ({"cache_kind": M.MIMO_CACHE_RING, "layer.window": 145, "ring_slots": 144}, M.MIMO_ERR_INVALID_ARG),
     ({"ring_slots": 100}, M.MIMO_ERR_INVALID_ARG),
     ({"ring_slots": 1024}, M.MIMO_ERR_INVALID_ARG),
+    ({"q_len": 9}, M.MIMO_ERR_INVALID_ARG),                                # beyond MIMO_MAX_DRAFTS
+    ({"q_len": -1}, M.MIMO_ERR_INVALID_ARG),
+    ({"q_len": 4, "max_seq_len": 3}, M.MIMO_ERR_INVALID_ARG),             # fewer positions than drafts
+    ({"q_len": 4, "workspace_bytes": 64}, M.MIMO_ERR_WORKSPACE),           # the draft route's partials
+    ({"q_len": 4, "workspace": None, "workspace_bytes": 0}, M.MIMO_ERR_WORKSPACE),
+    ({"q_len": 4, "cache_kind": M.MIMO_CACHE_RING, "layer.window": 128, "ring_slots": 128},
+     M.MIMO_ERR_INVALID_ARG),                                             # 128 + 4 - 1 keys > 128 slots
 ])
 def test_decode_validation(over, code):
     a = _decode_args(**over)
