@@ -24,6 +24,9 @@
 // softmax (exp2 domain, running max with rescale only when it grows by more
 // than 2^8, sink folded into the initial max and sum), write P into TMEM over
 // its S columns, and run the epilogue (O * v_scale / l -> bf16, LSE).
+// The global kernel also scores the draft rows of a decode on a paged cache (q_len rows
+// per sequence, no cu_seqlens): each sequence's keys are cut into page-aligned splits whose
+// partials the decode's combine pass merges.
 // Every wait is bounded: a wait that runs out sets MIMO_STATUS_TIMEOUT and the
 // CTA unwinds instead of hanging.
 #include <cuda_bf16.h>
